@@ -1,0 +1,543 @@
+"""Benchmark of the blockwise attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload flux] [--no-extra] [--no-cpu-baseline]
+
+One step is one pass of the hot path over one batch of the named workload:
+``pa_attn_fwd`` over each K/V chunk, then ``pa_attn_merge`` when the workload
+has more than one chunk.  The default workload is the FLUX-shaped joint
+attention (B=1, H=24, Nq=Nk=4608, d=128, one chunk).  The metric is attention
+forward TFLOPS, 4*B*H*Nq*Nk*d per step over the device time.
+
+Multi-GPU: one process per GPU (torchrun), every rank runs an independent
+replica of the step (the attention calls of different heads, batches or
+query blocks share nothing), so scaling is weak and there is no data-path
+collective; the process group only provides the barrier and the max over
+ranks of the timed region.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+on a bounded sample of the same workload instead (the reference arm).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "attention fwd TFLOPS (4·B·H·Nq·Nk·d/s) on 1 B200 and % of bf16 dense peak"
+UNIT = "TFLOPS"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of one attn_fwd launch on the default workload, from an ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
+# kernel source whose digest is recorded with it.  See profiles/.
+NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "capture": None}
+
+
+def _kernel_digest() -> str:
+    h = hashlib.sha256()
+    for f in ("ptx.cuh", "attn_fwd.cuh"):
+        with open(os.path.join(ROOT, "context_blocks_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# --------------------------------------------------------------------- clocks
+
+_REASONS = [(0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+            (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+            (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+            (0x100, "display_clock_setting")]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only)
+    from a thread while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - no NVML here
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((mhz, int(reasons)))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = [name for bit, name in _REASONS if mask & bit]
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
+
+
+# --------------------------------------------------------------- distributed
+
+def _dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over the default process group (identity
+    when no group is initialised)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(flops_per_step_per_rank: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOPS: the FLOPs all ranks processed over the slowest
+    rank's timed region."""
+    return flops_per_step_per_rank * steps * world / (max_ms * 1e-3) / 1e12
+
+
+# ------------------------------------------------------------------ our arm
+
+class Step:
+    """Buffers and launches of one hot-path step on one workload."""
+
+    def __init__(self, w: workloads.Workload, sets: int, device):
+        import torch
+        self.w = w
+        self.sets = []
+        n = len(w.chunks)
+        for s in range(sets):
+            q, k, v = workloads.make_case(w, device=device, seed=w.seed + 1000 * s)
+            pairs = workloads.split_keys(k, v, w.chunks)
+            del k, v
+            o = torch.empty_like(q)
+            lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+            o_parts = lse_parts = None
+            if n > 1:
+                o_parts = torch.empty((n,) + tuple(q.shape), dtype=torch.bfloat16, device=device)
+                lse_parts = torch.empty((n,) + tuple(q.shape[:3]), dtype=torch.float32, device=device)
+            self.sets.append((q, pairs, o, lse, o_parts, lse_parts))
+        self.launches_per_step = n + (1 if n > 1 else 0)
+
+    def bytes_resident(self) -> int:
+        tot = 0
+        for q, pairs, o, lse, op, lp in self.sets:
+            tot += q.numel() * 2 + sum(k.numel() * 4 for k, _ in pairs) + o.numel() * 2 + lse.numel() * 4
+            if op is not None:
+                tot += op.numel() * 2 + lp.numel() * 4
+        return tot
+
+    def run(self, i: int, pa, fwd_events=None, merge_events=None):
+        q, pairs, o, lse, o_parts, lse_parts = self.sets[i % len(self.sets)]
+        n = len(pairs)
+        for p, (k, v) in enumerate(pairs):
+            out = o if n == 1 else o_parts[p]
+            ls = lse if n == 1 else lse_parts[p]
+            if fwd_events is not None:
+                fwd_events[0].append(_record())
+            pa.attn_fwd(q, k, v, scale=self.w.scale, out=out, lse=ls)
+            if fwd_events is not None:
+                fwd_events[1].append(_record())
+        if n > 1:
+            if merge_events is not None:
+                merge_events[0].append(_record())
+            pa.attn_merge(o_parts, lse_parts, out=o, lse=lse)
+            if merge_events is not None:
+                merge_events[1].append(_record())
+
+
+def _record():
+    import torch
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()
+    return e
+
+
+def _sets_for(w: workloads.Workload) -> int:
+    per_set = workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk, w.d)
+    return max(1, min(8, math.ceil(2.5 * L2_BYTES / per_set)))
+
+
+def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None):
+    """Device time of `steps` steps (CUDA events on the launching stream,
+    synchronised on both sides).  Returns a dict of timings."""
+    import torch
+    st = Step(w, _sets_for(w), device)
+    for i in range(warmup):
+        st.run(i, pa)
+    torch.cuda.synchronize()
+    fwd_ev = ([], [])
+    mrg_ev = ([], [])
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        start.record()
+        for i in range(steps):
+            st.run(i, pa, fwd_ev, mrg_ev)
+        end.record()
+        torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = [a.elapsed_time(b) for a, b in zip(*fwd_ev)]
+    mrg_ms = [a.elapsed_time(b) for a, b in zip(*mrg_ev)]
+    status = pa.poll_device_status()
+    res = {"total_ms": total_ms, "fwd_ms": fwd_ms, "merge_ms": mrg_ms,
+           "launches": steps * st.launches_per_step, "sets": len(st.sets),
+           "resident_mb": st.bytes_resident() / 1e6, "status": status}
+    del st
+    torch.cuda.empty_cache()
+    return res
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def e2e_throughput(pa, w, steps, device):
+    """Same metric through the public API from pinned HOST buffers: every
+    step copies q and the K/V chunks host->device, runs the step, and copies
+    o and lse device->host; all inside the timed region."""
+    import torch
+    q, k, v = workloads.make_case(w, device=device)
+    pairs = workloads.split_keys(k, v, w.chunks)
+    hq = q.cpu().pin_memory()
+    hpairs = [(kk.cpu().pin_memory(), vv.cpu().pin_memory()) for kk, vv in pairs]
+    dq = torch.empty_like(q)
+    dpairs = [(torch.empty_like(kk), torch.empty_like(vv)) for kk, vv in pairs]
+    n = len(pairs)
+    B, H, Nq, d = q.shape
+    o_parts = torch.empty((n, B, H, Nq, d), dtype=torch.bfloat16, device=device) if n > 1 else None
+    lse_parts = torch.empty((n, B, H, Nq), dtype=torch.float32, device=device) if n > 1 else None
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=device)
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = hq.numel() * 2 + sum(a.numel() * 2 + b.numel() * 2 for a, b in hpairs)
+    d2h = ho.numel() * 2 + hl.numel() * 4
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        for (dk, dv), (hk, hv) in zip(dpairs, hpairs):
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+        pa.blockwise_attention(dq, [a for a, _ in dpairs], [b for _, b in dpairs], scale=w.scale,
+                               o_parts=o_parts, lse_parts=lse_parts, out=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        one()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
+    return {"value": fl * steps / (ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps}
+
+
+# ------------------------------------------------------------ CPU (oracle) leg
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 0) for i in info), default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_sample(w, seconds: float, seed_rows: int = 0):
+    """Time the oracle on a bounded sample of workload `w`: all heads and
+    batches, a prefix of `rows` query rows, every key of every chunk, chunks
+    merged as the GPU path does.  Rows are chosen from a short calibration
+    so that the sample takes about `seconds`.  Returns (tflops, seconds,
+    rows, description)."""
+    import numpy as np
+    import oracle
+    q, k, v = workloads.make_case(w, device="cpu", nq=min(w.Nq, 64))
+    qn = q.double().numpy()
+    kn, vn = k.double().numpy(), v.double().numpy()
+
+    def run(rows):
+        t0 = time.perf_counter()
+        qq = np.ascontiguousarray(np.resize(qn, (w.B, w.H, rows, w.d))) if rows > qn.shape[2] else qn[:, :, :rows]
+        if len(w.chunks) == 1:
+            oracle.attention(qq, kn, vn, w.scale)
+        else:
+            oracle.chunked_attention(qq, kn, vn, w.scale, w.chunks)
+        return time.perf_counter() - t0
+
+    cal_rows = 8
+    t_cal = max(run(cal_rows), 1e-4)
+    rows = int(max(1, min(w.Nq, cal_rows * seconds / t_cal)))
+    t = run(rows)
+    fl = workloads.flops(w.B, w.H, rows, w.Nk, w.d)
+    desc = (f"{w.name}: all {w.B}x{w.H} (batch x head) of {rows} query rows x {w.Nk} keys"
+            f"{' in ' + str(len(w.chunks)) + ' chunks + merge' if len(w.chunks) > 1 else ''}, fp64 NumPy")
+    return fl / t / 1e12, t, rows, desc
+
+
+# --------------------------------------------------------------------- main
+
+def _config(w, sets=None, resident_mb=None):
+    c = {"workload": f"{w.name}: B={w.B} H={w.H} Nq={w.Nq} Nk={w.Nk} d={w.d}, "
+                     f"{len(w.chunks)} K/V chunk(s) {list(w.chunks) if len(w.chunks) > 1 else ''}".strip(),
+         "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "chunks": list(w.chunks),
+         "parallelism": "replicas (one independent step per GPU)"}
+    if sets is not None:
+        c["l2"] = (f"inputs rotate over {sets} seeded sets, {resident_mb:.0f} MB resident "
+                   f"> 126 MB L2, so no step reads the previous step's inputs from L2")
+    return c
+
+
+def run_reference(args):
+    ws, rank, _ = _dist_env()
+    if rank != 0:
+        return 0
+    w = workloads.get(args.workload)
+    total_budget = args.cpu_budget
+    per_step = max(0.02, total_budget / max(1, args.steps + args.warmup))
+    tflops_cal, t_cal, rows, desc = oracle_sample(w, per_step)
+    fl_step = workloads.flops(w.B, w.H, rows, w.Nk, w.d)
+    import numpy as np
+    import oracle
+    q, k, v = workloads.make_case(w, device="cpu", nq=min(w.Nq, max(rows, 1)))
+    qn, kn, vn = q.double().numpy(), k.double().numpy(), v.double().numpy()
+    qn = np.ascontiguousarray(np.resize(qn, (w.B, w.H, rows, w.d))) if rows > qn.shape[2] else qn[:, :, :rows]
+
+    def step():
+        if len(w.chunks) == 1:
+            oracle.attention(qn, kn, vn, w.scale)
+        else:
+            oracle.chunked_attention(qn, kn, vn, w.scale, w.chunks)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = fl_step * args.steps / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    ws, rank, local = _dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    barrier = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        barrier = lambda: dist.barrier(device_ids=[local])  # noqa: E731
+    from context_blocks_b200 import build
+    if rank == 0:
+        build.build()
+    if barrier:
+        barrier()
+    import context_blocks_b200 as pa
+    pa.load_library()
+
+    w = workloads.get(args.workload)
+    peaks = _peaks()
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else local)
+    res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier)
+    if res["status"] != 0:
+        raise SystemExit(f"device status {res['status']} after the timed region")
+    max_ms = max_over_ranks(res["total_ms"], device)
+    fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
+    value = aggregate_throughput(fl, args.steps, ws, max_ms)
+
+    # Roofline of the dominant kernel (attn_fwd): algorithmic FLOPs per launch
+    # over its mean launch duration, against the measured bf16 dense peak.
+    fwd_mean_ms = statistics.fmean(res["fwd_ms"])
+    fl_launch = fl / len(w.chunks)
+    achieved = fl_launch / (fwd_mean_ms * 1e-3) / 1e12
+    traffic = None
+    if NCU_TRAFFIC["source_sha256"] == _kernel_digest():
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+            "kernel": "attn_fwd_kernel<128>", "launch_ms": fwd_mean_ms,
+            "peak_basis": f"{peaks['source']} burst bf16 (MEASURED_PEAKS.json bf16_tflops); "
+                          f"frac of sustained {achieved / peaks['bf16_tflops_sustained']:.3f}",
+            "algorithmic_bytes_per_launch": workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk // len(w.chunks), w.d)}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": _config(w, res["sets"], res["resident_mb"]),
+            "pct_of_bf16_peak": 100.0 * (value / ws) / peaks["bf16_tflops"],
+            "roofline": roof, "clocks": sampler.summary(), "gpu_launches": res["launches"]}
+    if res["merge_ms"]:
+        mb = workloads.merge_bytes(len(w.chunks), w.B, w.H, w.Nq, w.d)
+        line["merge"] = {"launch_ms": statistics.fmean(res["merge_ms"]),
+                         "gbs": mb / (statistics.fmean(res["merge_ms"]) * 1e-3) / 1e9,
+                         "peak_gbs": peaks["hbm_gbs"]}
+
+    if rank == 0 or ws > 1:
+        line["e2e"] = e2e_throughput(pa, w, steps=max(3, min(args.steps, 20)), device=device)
+        if ws > 1:
+            line["e2e"]["value"] = max_over_ranks(-line["e2e"]["value"], device) * -1 * ws
+
+    if ws == 1 and not args.no_extra:
+        line["extra"] = extra_measurements(pa, device, peaks)
+    if ws == 1 and not args.no_cpu_baseline:
+        tf, t, rows, desc = oracle_sample(w, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+                                "sample": desc, "seconds": t}
+    if barrier:
+        barrier()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def extra_measurements(pa, device, peaks):
+    """Secondary lines: the other workloads' device throughput (not the
+    headline value).  Bounded repetitions each."""
+    out = {}
+    plan = [("ring", 20, 3), ("tails", 10, 3), ("hunyuan", 3, 1)]
+    for name, steps, warm in plan:
+        w = workloads.get(name)
+        r = time_workload(pa, w, steps, warm, device)
+        fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
+        ent = {"step_ms": r["total_ms"] / steps, "tflops_step": fl * steps / (r["total_ms"] * 1e-3) / 1e12,
+               "fwd_ms_per_launch": statistics.fmean(r["fwd_ms"]),
+               "fwd_tflops": (fl / len(w.chunks)) / (statistics.fmean(r["fwd_ms"]) * 1e-3) / 1e12}
+        if r["merge_ms"]:
+            mb = workloads.merge_bytes(len(w.chunks), w.B, w.H, w.Nq, w.d)
+            ent["merge_ms"] = statistics.fmean(r["merge_ms"])
+            ent["merge_gbs"] = mb / (ent["merge_ms"] * 1e-3) / 1e9
+        ent["pct_of_bf16_peak"] = 100.0 * ent["fwd_tflops"] / peaks["bf16_tflops"]
+        out[name] = ent
+    w8 = workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8)
+    r = time_workload(pa, w8, 2, 1, device)
+    fl = workloads.flops(w8.B, w8.H, w8.Nq, w8.Nk, w8.d)
+    mb = workloads.merge_bytes(8, w8.B, w8.H, w8.Nq, w8.d)
+    out["hunyuan_8chunks"] = {"step_ms": r["total_ms"] / 2,
+                              "tflops_step": fl * 2 / (r["total_ms"] * 1e-3) / 1e12,
+                              "fwd_tflops": (fl / 8) / (statistics.fmean(r["fwd_ms"]) * 1e-3) / 1e12,
+                              "merge_ms": statistics.fmean(r["merge_ms"]),
+                              "merge_gbs": mb / (statistics.fmean(r["merge_ms"]) * 1e-3) / 1e9}
+    return out
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="flux", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU seconds of the oracle sample in the cpu_baseline leg")
+    ap.add_argument("--cpu-budget", type=float, default=120.0,
+                    help="total CPU seconds of the reference arm's timed steps")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,19 @@
+"""Blockwise (ring-step) attention for NVIDIA B200, as a C-ABI CUDA library.
+
+``attn_fwd`` attends every query row to one K/V chunk and returns the
+normalised partial output with its natural log-sum-exp; ``attn_merge``
+combines partial results over disjoint chunks into the exact full result;
+``blockwise_attention`` chains the two over a list of chunks.  The kernels
+live in ``libpa_attn.so`` (``include/pa_attn.h``); this package only loads it
+and marshals arguments.  Build it with ``python -m context_blocks_b200.build``.
+"""
+
+from ._binding import (LIB_PATH, PA_ERR_CUDA, PA_ERR_INVALID_ARG, PA_ERR_MISALIGNED, PA_ERR_TIMEOUT,
+                       PA_ERR_UNSUPPORTED, PA_OK, PaError, attn_fwd, attn_merge, last_error,
+                       load_library, poll_device_status, selftest_timeout, status_string, version)
+from .ring import blockwise_attention
+
+__all__ = ["LIB_PATH", "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_MISALIGNED",
+           "PA_ERR_CUDA", "PA_ERR_TIMEOUT", "PaError", "attn_fwd", "attn_merge",
+           "blockwise_attention", "last_error", "load_library", "poll_device_status",
+           "selftest_timeout", "status_string", "version"]

@@ -1,0 +1,177 @@
+"""ctypes binding of ``libpa_attn.so`` (the C ABI in ``include/pa_attn.h``).
+
+Argument marshalling only: tensors are checked for dtype, device, layout and
+shape, their device pointers and sizes are handed to the C entry points, and
+a non-zero status becomes a :class:`PaError`.  Every step of the attention
+and the merge runs in the library's CUDA kernels.  There is no fallback: if
+the library is missing or does not load, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libpa_attn.so")
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = -1
+PA_ERR_UNSUPPORTED = -2
+PA_ERR_MISALIGNED = -3
+PA_ERR_CUDA = -4
+PA_ERR_TIMEOUT = -5
+
+# (name, restype, argtypes) for every symbol declared in include/pa_attn.h.
+_VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "pa_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
+    "pa_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _VP]),
+    "pa_status_string": (ctypes.c_char_p, [_I]),
+    "pa_last_error": (ctypes.c_char_p, []),
+    "pa_poll_device_status": (_I, []),
+    "pa_selftest_timeout": (_I, [_I, _VP]),
+    "pa_version": (_I, []),
+}
+
+
+class PaError(RuntimeError):
+    """A non-zero status from the C library."""
+
+    def __init__(self, code: int, where: str, detail: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({detail})" if detail else
+                         f"{where}: {status_string(code)}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load (once) and return the library; raises if it is not built."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is missing: build it with `python -m context_blocks_b200.build`")
+        lib = ctypes.CDLL(p)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().pa_status_string(int(code)).decode()
+
+
+def last_error() -> str:
+    return load_library().pa_last_error().decode()
+
+
+def version() -> int:
+    return int(load_library().pa_version())
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != PA_OK:
+        raise PaError(rc, where, last_error())
+
+
+def _stream_handle(stream, device) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def _check_bf16(name, t, ndim):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16 (got {t.dtype})")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must live on a CUDA device")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """Attention of q [B,H,Nq,d] against one K/V chunk k, v [B,H,Nk,d].
+
+    Returns (o [B,H,Nq,d] bf16, lse [B,H,Nq] fp32, natural log), written into
+    ``out`` / ``lse`` when given.  ``scale`` defaults to 1/sqrt(d).
+    """
+    import torch
+    _check_bf16("q", q, 4)
+    _check_bf16("k", k, 4)
+    _check_bf16("v", v, 4)
+    B, H, Nq, d = q.shape
+    if k.shape[:2] != (B, H) or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_bf16("out", out, 4)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B,H,Nq] tensor")
+    rc = load_library().pa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, H, Nq, Nk, d, float(scale),
+                                    _stream_handle(stream, q.device))
+    _check(rc, "pa_attn_fwd")
+    return out, lse
+
+
+def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
+    """Merge n partial results o_parts [n,B,H,N,d] bf16, lse_parts [n,B,H,N]
+    fp32 (over disjoint key chunks) into (o [B,H,N,d], lse [B,H,N])."""
+    import torch
+    _check_bf16("o_parts", o_parts, 5)
+    n, B, H, N, d = o_parts.shape
+    if (lse_parts.dtype != torch.float32 or tuple(lse_parts.shape) != (n, B, H, N)
+            or not lse_parts.is_contiguous() or lse_parts.device != o_parts.device):
+        raise ValueError("lse_parts must be a contiguous float32 [n,B,H,N] tensor on o_parts' device")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=o_parts.device)
+    else:
+        _check_bf16("out", out, 4)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=o_parts.device)
+    rc = load_library().pa_attn_merge(o_parts.data_ptr(), lse_parts.data_ptr(), n, out.data_ptr(),
+                                      lse.data_ptr(), B, H, N, d,
+                                      _stream_handle(stream, o_parts.device))
+    _check(rc, "pa_attn_merge")
+    return out, lse
+
+
+def poll_device_status() -> int:
+    """Read and clear the device status word (synchronising).  Returns the
+    status code (0 = no device-side error since the last poll)."""
+    return int(load_library().pa_poll_device_status())
+
+
+def selftest_timeout(limit_us: int, stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (see pa_selftest_timeout)."""
+    import torch
+    rc = load_library().pa_selftest_timeout(int(limit_us),
+                                            _stream_handle(stream, torch.cuda.current_device()))
+    _check(rc, "pa_selftest_timeout")

@@ -1,0 +1,397 @@
+// Blockwise attention forward for one K/V chunk on sm_100a.
+//
+// Computes, for every (b, h) and query row i of this call,
+//     O_i   = sum_j softmax_j(scale * q_i . k_j) v_j        (normalised)
+//     LSE_i = ln sum_j exp(scale * q_i . k_j)               (natural log)
+// over the keys j of the chunk given to the call.  This is the per-block
+// step of Ring Attention as the diffusers "Context parallelism" guide
+// describes it (section "Ring Attention": each device attends with the K/V
+// block it holds); the (O, LSE) pair is what the merge kernel needs to
+// combine blocks into the exact full-sequence result.  Keys past the chunk's
+// real length never enter the softmax (section "Ring Anything Attention":
+// blocks are trimmed back to their real length before attention).
+//
+// Kernel structure (one CTA per 256 query rows of one (b, h)):
+//   warps 0-3  softmax warpgroup for query tile 0 (rows   0..127 of the block)
+//   warps 4-7  softmax warpgroup for query tile 1 (rows 128..255 of the block)
+//   warp  8    TMEM allocation + single-thread tcgen05.mma issue
+//   warp  9    single-thread TMA producer (Q once, then K_j / V_j ring)
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [0,128)        S_0 = Q_0 K_j^T   (P_0 is written back over it as bf16)
+//   [128,256)      S_1 = Q_1 K_j^T   (P_1 likewise)
+//   [256,256+D)    O_0 accumulator
+//   [256+D,256+2D) O_1 accumulator
+// Thread t of softmax warpgroup i owns TMEM lane t = query row t of tile i,
+// so row max, row sum and rescaling need no cross-thread reduction.
+//
+// Online softmax in base 2: x = s * scale * log2(e).  m_ref is the reference
+// maximum the exponentials of this row use; it moves only when a new tile's
+// maximum exceeds it by more than kRescaleLog2 (lazy rescaling), in which case
+// the running sum l and the O accumulator are multiplied by
+// 2^(m_ref_old - m_ref_new).  Unnormalised P = 2^(x - m_ref) <= 2^kRescaleLog2.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace pa {
+
+constexpr int kBM = 128;           // query rows per tile (= TMEM lanes)
+constexpr int kBN = 128;           // keys per K/V tile
+constexpr int kQTiles = 2;         // query tiles per CTA
+constexpr int kStages = 4;         // K/V ring slots (each holds one K or one V tile)
+constexpr int kFwdThreads = 320;   // 10 warps
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+// Device status codes written by kernels (mirror PA_ERR_* in pa_attn.h).
+constexpr int kStatusTimeout = -5;
+
+template <int D>
+struct FwdLayout {
+  static_assert(D == 64 || D == 128, "head dim must be 64 or 128");
+  static constexpr int kBoxBytes = 128 * 128;        // 128 rows x 64 bf16, 128B-swizzled
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row tile of Q, K or V
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = kQOff + kQTiles * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  // q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kAbortOff = kTmemSlotOff + 4;
+  static constexpr int kBytes = kAbortOff + 4;
+  // Slack to align the base to 1024 B.  The request is also padded so that a
+  // second CTA never fits on the SM: each CTA takes all 512 TMEM columns, and
+  // a co-resident CTA would only sit blocked in tcgen05.alloc.
+  static constexpr int kMinOneCtaPerSm = 120 * 1024;
+  static constexpr int kAllocBytes =
+      (kBytes + 1024 > kMinOneCtaPerSm) ? (kBytes + 1024) : kMinOneCtaPerSm;
+};
+
+struct FwdParams {
+  __nv_bfloat16* o;     // [B*H, Nq, D]
+  float* lse;           // [B*H, Nq]
+  int Nq;
+  int Nk;
+  int n_kv_tiles;       // ceil(Nk / kBN)
+  float scale_log2;     // scale * log2(e)
+  int* status;          // device status word
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const uint32_t sQ = base + L::kQOff;
+  const uint32_t sRing = base + L::kRingOff;
+  const uint32_t bars = base + L::kBarOff;
+  const uint32_t bar_q_full0 = bars;
+  const uint32_t bar_kv_full0 = bars + 8 * 2;
+  const uint32_t bar_kv_empty0 = bars + 8 * (2 + kStages);
+  const uint32_t bar_s_full0 = bars + 8 * (2 + 2 * kStages);
+  const uint32_t bar_p_full0 = bars + 8 * (4 + 2 * kStages);
+  const uint32_t bar_o_full0 = bars + 8 * (6 + 2 * kStages);
+  const uint32_t bar_drain = bars + 8 * (8 + 2 * kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kTmemSlotOff);
+  volatile int* abort_word = reinterpret_cast<volatile int*>(gbase + L::kAbortOff);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int q0 = blockIdx.x * (kQTiles * kBM);
+  const int bh = blockIdx.y;
+  const int n = p.n_kv_tiles;
+  const uint64_t lim = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) mbar_init(bar_q_full0 + 8 * i, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_kv_full0 + 8 * s, 1);
+      mbar_init(bar_kv_empty0 + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_s_full0 + 8 * i, 1);
+      mbar_init(bar_p_full0 + 8 * i, 4);  // one arrival per softmax warp
+      mbar_init(bar_o_full0 + 8 * i, 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_word = 0;
+    fence_barrier_init();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int i = 0; i < kQTiles; ++i) {
+        mbar_arrive_expect_tx(bar_q_full0 + 8 * i, L::kTileBytes);
+#pragma unroll
+        for (int b = 0; b < L::kBoxes; ++b)
+          tma_load_3d(sQ + i * L::kTileBytes + b * L::kBoxBytes, &tm_q, bar_q_full0 + 8 * i, b * 64,
+                      q0 + i * kBM, bh);
+      }
+      bool ok = true;
+      int idx = 0;  // ring loads issued so far
+      for (int j = 0; j < n && ok; ++j) {
+        for (int t = 0; t < 2; ++t) {  // t = 0: K_j, t = 1: V_j
+          const int s = idx % kStages;
+          const uint32_t u = idx / kStages;
+          if (!mbar_wait(bar_kv_empty0 + 8 * s, (u & 1) ^ 1, abort_word, p.status, kStatusTimeout, lim)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = bar_kv_full0 + 8 * s;
+          mbar_arrive_expect_tx(full, L::kTileBytes);
+          const CUtensorMap* map = t ? &tm_v : &tm_k;
+#pragma unroll
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_3d(sRing + s * L::kTileBytes + b * L::kBoxBytes, map, full, b * 64, j * kBN, bh);
+          ++idx;
+        }
+      }
+      if (!ok) {
+        // Aborted: let every copy already in flight land before the CTA exits.
+        // Slot s received ceil((idx - s) / kStages) loads; wait for the last.
+        for (int i = 0; i < kQTiles; ++i)
+          mbar_wait(bar_q_full0 + 8 * i, 0, nullptr, p.status, kStatusTimeout, lim);
+        for (int s = 0; s < kStages && s < idx; ++s) {
+          const int cnt = (idx - s + kStages - 1) / kStages;
+          mbar_wait(bar_kv_full0 + 8 * s, (cnt - 1) & 1, nullptr, p.status, kStatusTimeout, lim);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(128, kBN, false, false);
+      constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
+      const uint32_t tO0 = tmem + 2 * kBN;
+
+      // S_i = Q_i K^T : K-major Q and K, 16 bf16 of depth per instruction.
+      auto issue_qk = [&](int i, uint32_t sK) {
+        const uint32_t sq = sQ + i * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * L::kBoxBytes + (kk % 4) * 32;
+          umma_ss(tmem + i * kBN, sdesc_k_sw128(sq + off), sdesc_k_sw128(sK + off), kIdS, kk > 0);
+        }
+      };
+      // O_i (+)= P_i V : P from TMEM (bf16 pairs, 8 columns per 16 keys),
+      // V MN-major (rows of 64 head-dim elements, 16 keys = 2048 bytes).
+      auto issue_pv = [&](int i, uint32_t sV, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts(tO0 + i * D, tmem + i * kBN + kk * 8, sdesc_mn_sw128(sV + kk * 2048, L::kBoxBytes),
+                  kIdPV, (acc || kk > 0) ? 1u : 0u);
+      };
+
+      bool ok = mbar_wait(bar_q_full0, 0, abort_word, p.status, kStatusTimeout, lim) &&
+                mbar_wait(bar_q_full0 + 8, 0, abort_word, p.status, kStatusTimeout, lim) &&
+                mbar_wait(bar_kv_full0, 0, abort_word, p.status, kStatusTimeout, lim);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, sRing);
+        umma_commit(bar_s_full0);
+        issue_qk(1, sRing);
+        umma_commit(bar_s_full0 + 8);
+        umma_commit(bar_kv_empty0);
+      }
+      int idx = 1;
+      for (int j = 0; j < n && ok; ++j) {
+        const int sv = idx % kStages;
+        const uint32_t uv = idx / kStages;
+        ++idx;
+        int sk = 0;
+        uint32_t uk = 0;
+        const bool more = (j + 1 < n);
+        if (more) {
+          sk = idx % kStages;
+          uk = idx / kStages;
+          ++idx;
+        }
+        if (!mbar_wait(bar_kv_full0 + 8 * sv, uv & 1, abort_word, p.status, kStatusTimeout, lim)) {
+          ok = false;
+          break;
+        }
+        for (int i = 0; i < 2; ++i) {
+          if (!mbar_wait(bar_p_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(i, sRing + sv * L::kTileBytes, j > 0);
+          if (i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
+          if (more) {
+            if (i == 0) {
+              if (!mbar_wait(bar_kv_full0 + 8 * sk, uk & 1, abort_word, p.status, kStatusTimeout, lim)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            issue_qk(i, sRing + sk * L::kTileBytes);
+            umma_commit(bar_s_full0 + 8 * i);
+            if (i == 1) umma_commit(bar_kv_empty0 + 8 * sk);
+          } else {
+            umma_commit(bar_o_full0 + 8 * i);
+          }
+        }
+      }
+      // Every MMA this thread issued completes before tensor memory is freed.
+      umma_commit(bar_drain);
+      mbar_wait(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int i = warp / 4;                    // query tile of this warpgroup
+    const int t = threadIdx.x % 128;           // row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + i * kBN + lane_off;
+    const uint32_t tO = tmem + 2 * kBN + i * D + lane_off;
+    const int row = q0 + i * kBM + t;
+    const float c = p.scale_log2;
+    float m_ref = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+
+    for (int j = 0; j < n; ++j) {
+      const bool got = mbar_wait(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim);
+      if (__any_sync(0xffffffffu, !got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[kBN];
+      tmem_ld_x128(tS, sr);
+      float s[kBN];
+#pragma unroll
+      for (int e = 0; e < kBN; ++e) s[e] = __uint_as_float(sr[e]);
+      const int valid = p.Nk - j * kBN;  // keys of this tile inside the chunk
+      if (valid < kBN) {
+#pragma unroll
+        for (int e = 0; e < kBN; ++e)
+          if (e >= valid) s[e] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int e = 1; e < kBN; ++e) mx = fmaxf(mx, s[e]);
+      mx *= c;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mx > m_ref + kRescaleLog2) {
+        alpha = ex2_approx(m_ref - mx);  // 0 on the first tile (m_ref = -inf)
+        l *= alpha;
+        m_ref = mx;
+        rescale = (j > 0);
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // PV of tile j-1 has completed: S_i(j) was issued after it and the
+        // tcgen05 ops of the issuing thread complete in order.
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t orr[32];
+          tmem_ld_x32(tO + ch * 32, orr);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+          tmem_st_x32(tO + ch * 32, orr);
+        }
+      }
+      const float neg_m = -m_ref;
+#pragma unroll
+      for (int ch = 0; ch < kBN / 32; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(s[ch * 32 + 2 * e], c, neg_m));
+          const float p1 = ex2_approx(fmaf(s[ch * 32 + 2 * e + 1], c, neg_m));
+          l += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_x16(tS + ch * 16, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full0 + 8 * i);
+    }
+
+    if (ok) {
+      const bool got = mbar_wait(bar_o_full0 + 8 * i, 0, abort_word, p.status, kStatusTimeout, lim);
+      ok = !__any_sync(0xffffffffu, !got);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool in_range = row < p.Nq;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.Nq + row) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t orr[32];
+        tmem_ld_x32(tO + ch * 32, orr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (in_range)
+        p.lse[static_cast<size_t>(bh) * p.Nq + row] = (m_ref + lg2_approx(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,324 @@
+// C ABI of the blockwise attention library: argument checks, TMA tensor-map
+// encoding and kernel launches.  See include/pa_attn.h for the contract.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "attn_fwd.cuh"
+#include "lse_merge.cuh"
+#include "pa_attn.h"
+
+namespace pa {
+
+// Device status word: kernels record the first device-side error here.
+__device__ int g_status = 0;
+
+__global__ void timeout_probe_kernel(unsigned long long limit_ns, int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_word = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`; the bounded wait gives up after limit_ns.
+  mbar_wait(smem_u32(&bar), 0, &abort_word, status, kStatusTimeout, limit_ns);
+}
+
+}  // namespace pa
+
+namespace {
+
+constexpr unsigned long long kDefaultTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s
+constexpr int kMaxDevices = 64;
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(PA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+struct DeviceState {
+  bool ready = false;
+  bool supported = false;
+  int sm_count = 0;
+  int* status = nullptr;  // device address of pa::g_status
+  bool fwd_attr[2] = {false, false};
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+// Per-device set-up, once: capability check, SM count, status-word address.
+int device_state(int dev, DeviceState** out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    int major = 0, minor = 0, sms = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    s.supported = (major == 10 && minor == 0);
+    s.sm_count = sms;
+    if (s.supported) {
+      void* addr = nullptr;
+      e = cudaGetSymbolAddress(&addr, pa::g_status);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+      s.status = static_cast<int*>(addr);
+    }
+    s.ready = true;
+  }
+  if (!s.supported) return fail(PA_ERR_UNSUPPORTED, "device %d is not sm_100 (B200)", dev);
+  *out = &s;
+  return PA_OK;
+}
+
+// The pointer must be device (or managed) memory of the current device.
+int check_device_ptr(const void* ptr, const char* name, int* dev_out) {
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, ptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return fail(PA_ERR_INVALID_ARG, "%s is not device memory", name);
+  int cur = 0;
+  e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (attr.device != cur)
+    return fail(PA_ERR_INVALID_ARG, "%s lives on device %d, current device is %d", name, attr.device, cur);
+  *dev_out = cur;
+  return PA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, uint64_t na, const void* b, uint64_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a [BH, N, d] bf16 tensor: box of 64 head-dim elements x 128
+// rows x 1, 128-byte swizzle, zero fill outside the tensor.
+int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n_rows),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(n_rows) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(pa::kBM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+  return PA_OK;
+}
+
+template <int D>
+int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int BH,
+               int Nq, int Nk, float scale, cudaStream_t stream) {
+  using L = pa::FwdLayout<D>;
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = encode_map(&tq, q, D, Nq, BH)) != PA_OK) return rc;
+  if ((rc = encode_map(&tk, k, D, Nk, BH)) != PA_OK) return rc;
+  if ((rc = encode_map(&tv, v, D, Nk, BH)) != PA_OK) return rc;
+  auto kern = pa::attn_fwd_kernel<D>;
+  const int slot = (D == 64) ? 0 : 1;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!st->fwd_attr[slot]) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      st->fwd_attr[slot] = true;
+    }
+  }
+  pa::FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.n_kv_tiles = (Nk + pa::kBN - 1) / pa::kBN;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.status = st->status;
+  prm.timeout_ns = kDefaultTimeoutNs;
+  dim3 grid((Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM), BH);
+  kern<<<grid, pa::kFwdThreads, L::kAllocBytes, stream>>>(tq, tk, tv, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
+  return PA_OK;
+}
+
+template <int D>
+int launch_merge(DeviceState* st, const void* o_parts, const float* lse_parts, int n_parts, void* o,
+                 float* lse, long long rows, cudaStream_t stream) {
+  constexpr int kRpb = pa::kMergeThreads / (D / 8);
+  long long blocks = (rows + kRpb - 1) / kRpb;
+  const long long cap = static_cast<long long>(st->sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  pa::lse_merge_kernel<D><<<static_cast<unsigned>(blocks), pa::kMergeThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o_parts), lse_parts, n_parts, static_cast<__nv_bfloat16*>(o), lse,
+      rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "lse_merge launch");
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                int Nk, int d, float scale, void* stream) {
+  g_err[0] = '\0';
+  if (!q || !k || !v || !o || !lse) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (B < 1 || H < 1) return fail(PA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
+  if (Nq < 0) return fail(PA_ERR_INVALID_ARG, "Nq must be >= 0 (got %d)", Nq);
+  if (Nk < 1) return fail(PA_ERR_INVALID_ARG, "Nk must be >= 1 (got %d)", Nk);
+  if (!std::isfinite(scale) || !(scale > 0.f)) return fail(PA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (d != 64 && d != 128) return fail(PA_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > 65535) return fail(PA_ERR_UNSUPPORTED, "B*H must be <= 65535 (got %lld)", bh);
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+    return fail(PA_ERR_MISALIGNED, "q, k, v and o must be 16-byte aligned");
+  if (!aligned(lse, 4)) return fail(PA_ERR_MISALIGNED, "lse must be 4-byte aligned");
+  if (Nq == 0) return PA_OK;
+  const uint64_t qbytes = static_cast<uint64_t>(bh) * Nq * d * 2;
+  const uint64_t kbytes = static_cast<uint64_t>(bh) * Nk * d * 2;
+  const uint64_t lbytes = static_cast<uint64_t>(bh) * Nq * 4;
+  const void* ins[3] = {q, k, v};
+  const uint64_t in_bytes[3] = {qbytes, kbytes, kbytes};
+  for (int i = 0; i < 3; ++i)
+    if (overlap(ins[i], in_bytes[i], o, qbytes) || overlap(ins[i], in_bytes[i], lse, lbytes))
+      return fail(PA_ERR_INVALID_ARG, "outputs overlap an input");
+  if (overlap(o, qbytes, lse, lbytes)) return fail(PA_ERR_INVALID_ARG, "o and lse overlap");
+
+  (void)cudaGetLastError();
+  int dev = 0, rc;
+  const void* ptrs[5] = {q, k, v, o, lse};
+  const char* names[5] = {"q", "k", "v", "o", "lse"};
+  for (int i = 0; i < 5; ++i)
+    if ((rc = check_device_ptr(ptrs[i], names[i], &dev)) != PA_OK) return rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(dev, &st)) != PA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_fwd<64>(st, q, k, v, o, lse, static_cast<int>(bh), Nq, Nk, scale, s);
+  return launch_fwd<128>(st, q, k, v, o, lse, static_cast<int>(bh), Nq, Nk, scale, s);
+}
+
+int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void* o, float* lse, int B, int H,
+                  int N, int d, void* stream) {
+  g_err[0] = '\0';
+  if (!o_parts || !lse_parts || !o || !lse) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (n_parts < 1) return fail(PA_ERR_INVALID_ARG, "n_parts must be >= 1 (got %d)", n_parts);
+  if (B < 1 || H < 1) return fail(PA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
+  if (N < 0) return fail(PA_ERR_INVALID_ARG, "N must be >= 0 (got %d)", N);
+  if (d != 64 && d != 128) return fail(PA_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  if (!aligned(o_parts, 16) || !aligned(o, 16))
+    return fail(PA_ERR_MISALIGNED, "o_parts and o must be 16-byte aligned");
+  if (!aligned(lse_parts, 4) || !aligned(lse, 4))
+    return fail(PA_ERR_MISALIGNED, "lse_parts and lse must be 4-byte aligned");
+  if (N == 0) return PA_OK;
+  const long long rows = static_cast<long long>(B) * H * N;
+  const uint64_t obytes = static_cast<uint64_t>(rows) * d * 2;
+  const uint64_t lbytes = static_cast<uint64_t>(rows) * 4;
+  if (overlap(o_parts, obytes * n_parts, o, obytes) || overlap(o_parts, obytes * n_parts, lse, lbytes) ||
+      overlap(lse_parts, lbytes * n_parts, o, obytes) || overlap(lse_parts, lbytes * n_parts, lse, lbytes) ||
+      overlap(o, obytes, lse, lbytes))
+    return fail(PA_ERR_INVALID_ARG, "outputs overlap an input");
+
+  (void)cudaGetLastError();
+  int dev = 0, rc;
+  const void* ptrs[4] = {o_parts, lse_parts, o, lse};
+  const char* names[4] = {"o_parts", "lse_parts", "o", "lse"};
+  for (int i = 0; i < 4; ++i)
+    if ((rc = check_device_ptr(ptrs[i], names[i], &dev)) != PA_OK) return rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(dev, &st)) != PA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_merge<64>(st, o_parts, lse_parts, n_parts, o, lse, rows, s);
+  return launch_merge<128>(st, o_parts, lse_parts, n_parts, o, lse, rows, s);
+}
+
+const char* pa_status_string(int code) {
+  switch (code) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: invalid argument";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: unsupported shape or device";
+    case PA_ERR_MISALIGNED: return "PA_ERR_MISALIGNED: pointer alignment";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime or driver error";
+    case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT: a device-side bounded wait gave up";
+    default: return "unknown status code";
+  }
+}
+
+const char* pa_last_error(void) { return g_err; }
+
+int pa_poll_device_status(void) {
+  g_err[0] = '\0';
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  DeviceState* st = nullptr;
+  int rc = device_state(dev, &st);
+  if (rc != PA_OK) return rc;
+  int value = 0;
+  e = cudaMemcpy(&value, st->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  const int zero = 0;
+  e = cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+  return value;
+}
+
+int pa_selftest_timeout(int limit_us, void* stream) {
+  g_err[0] = '\0';
+  if (limit_us < 1 || limit_us > 1000000) return fail(PA_ERR_INVALID_ARG, "limit_us must be in [1, 1e6]");
+  (void)cudaGetLastError();
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  DeviceState* st = nullptr;
+  int rc = device_state(dev, &st);
+  if (rc != PA_OK) return rc;
+  pa::timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull, st->status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "timeout probe launch");
+  return PA_OK;
+}
+
+int pa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+/*
+ * pa_attn.h - blockwise (ring-step) attention for NVIDIA B200 (sm_100a).
+ *
+ * A C ABI over two CUDA kernels:
+ *
+ *   pa_attn_fwd    attention of every query row against ONE key/value chunk,
+ *                  returning the normalised partial output O and the natural
+ *                  log-sum-exp LSE of the scaled logits over that chunk;
+ *   pa_attn_merge  the exact combination of n such partial results, computed
+ *                  over disjoint key chunks, into the full-sequence result.
+ *
+ * Together they are the per-device step of Ring Attention as the diffusers
+ * guide "Context parallelism" describes it (section "Ring Attention": each
+ * device attends with the K/V block it holds and passes the block on; after a
+ * full turn every device has seen the K/V of every token).  Chunks of any
+ * length are accepted (section "Ring Anything Attention": blocks are trimmed
+ * to their real length before attention, so padding never enters the
+ * softmax).  Attention is the non-causal, unmasked scaled-dot-product
+ * attention of the guide "Accelerate inference" (section "Scaled dot product
+ * attention"; inference only, attn_mask None), computed on bf16 inputs (same
+ * guide, section "Model data type") with fp32 accumulation.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Layouts are contiguous, row-major, head dimension innermost:
+ *     q, o   [B, H, Nq, d] bf16          k, v   [B, H, Nk, d] bf16
+ *     lse    [B, H, Nq]    fp32, natural log
+ * - All tensor pointers are DEVICE pointers on the current CUDA device, owned
+ *   and allocated by the caller.  The library allocates no memory in any call.
+ *   Inputs and outputs must not overlap.
+ * - q, k, v, o and o_parts must be 16-byte aligned (TMA / vector access);
+ *   lse and lse_parts 4-byte aligned.
+ * - d must be 64 or 128.
+ * - `stream` is a cudaStream_t (0 = legacy default stream).  Calls are fully
+ *   asynchronous: they validate arguments on the host, enqueue kernels on
+ *   `stream` and return.  They never synchronise the host and never copy
+ *   between host and device.
+ * - Return values: PA_OK or a negative PA_ERR_* code for errors the host can
+ *   see before or at launch.  Errors raised later on the device (a bounded
+ *   wait that gave up) are reported by pa_poll_device_status().
+ */
+#ifndef PA_ATTN_H_
+#define PA_ATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define PA_OK 0
+#define PA_ERR_INVALID_ARG (-1) /* null pointer, size out of range, non-finite or non-positive scale,
+                                   host (non-device) pointer, overlapping input/output */
+#define PA_ERR_UNSUPPORTED (-2) /* d not in {64, 128}, device not sm_100, B*H > 65535 */
+#define PA_ERR_MISALIGNED (-3)  /* a pointer breaks the alignment rule above */
+#define PA_ERR_CUDA (-4)        /* CUDA runtime / driver error; see pa_last_error() */
+#define PA_ERR_TIMEOUT (-5)     /* a device-side bounded wait gave up (from pa_poll_device_status) */
+
+/*
+ * pa_attn_fwd - attention of Q against one K/V chunk.
+ *
+ * For each b < B, h < H and query row i < Nq, over the keys j < Nk of the
+ * chunk (diffusers "Context parallelism", section "Ring Attention"):
+ *     s_ij    = scale * sum_c q[b,h,i,c] k[b,h,j,c]
+ *     lse[i]  = ln sum_j exp(s_ij)
+ *     o[i,:]  = sum_j exp(s_ij - lse[i]) v[b,h,j,:]        (rounded to bf16)
+ *
+ * q      [B,H,Nq,d] bf16, device, 16-byte aligned       (input)
+ * k, v   [B,H,Nk,d] bf16, device, 16-byte aligned       (input)
+ * o      [B,H,Nq,d] bf16, device, 16-byte aligned       (output, fully written)
+ * lse    [B,H,Nq]   fp32, device, 4-byte aligned        (output, fully written)
+ * B, H   >= 1, B*H <= 65535
+ * Nq     >= 0 (0 is a no-op returning PA_OK); Nk >= 1 (an empty chunk has no
+ *        attention: pass it to pa_attn_merge with lse = -inf instead)
+ * d      64 or 128
+ * scale  finite and > 0 (typically 1/sqrt(d))
+ * stream cudaStream_t
+ *
+ * Errors: PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_MISALIGNED before
+ * anything is enqueued; PA_ERR_CUDA if the launch fails.
+ */
+int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int Nq, int Nk, int d, float scale, void* stream);
+
+/*
+ * pa_attn_merge - combine n partial results over disjoint key chunks.
+ *
+ * For every row r of the B*H*N rows (same section as above: the per-block
+ * results combine into the exact full attention):
+ *     M = max_p lse_parts[p,r];  w_p = exp(lse_parts[p,r] - M);  L = sum_p w_p
+ *     o[r,:] = sum_p w_p o_parts[p,r,:] / L;     lse[r] = M + ln L
+ * A part with lse = -inf carries no weight and its o_parts row is not read;
+ * a row whose parts are all -inf gets o = 0 and lse = -inf.  n_parts = 1 is a
+ * copy.
+ *
+ * o_parts   [n_parts,B,H,N,d] bf16, device, 16-byte aligned   (input)
+ * lse_parts [n_parts,B,H,N]   fp32, device, 4-byte aligned    (input)
+ * o         [B,H,N,d] bf16, device, 16-byte aligned           (output)
+ * lse       [B,H,N]   fp32, device, 4-byte aligned            (output)
+ * n_parts >= 1; B, H >= 1; N >= 0 (0 is a no-op); d 64 or 128.
+ *
+ * Errors: as pa_attn_fwd.
+ */
+int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void* o, float* lse,
+                  int B, int H, int N, int d, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* pa_status_string(int code);
+
+/*
+ * Detail of the last PA_ERR_* returned on the calling host thread (the CUDA
+ * error string for PA_ERR_CUDA, the failed check otherwise).  The pointer
+ * stays valid until the next library call on this thread.
+ */
+const char* pa_last_error(void);
+
+/*
+ * Read and clear the device status word of the current device.  Kernels set
+ * it (first error wins) when a bounded wait inside them gives up; the kernel
+ * then releases its resources and exits instead of hanging.  Returns PA_OK,
+ * PA_ERR_TIMEOUT, or PA_ERR_CUDA if the word could not be read.  This call
+ * synchronises with the device (it copies 4 bytes device -> host): call it
+ * after the work of interest has completed, never on a hot path.
+ */
+int pa_poll_device_status(void);
+
+/*
+ * Exercise the bounded-wait path on the device: launch one CTA that waits on
+ * a shared-memory barrier nothing will ever complete, with a limit of
+ * `limit_us` microseconds (1 .. 1000000).  The wait gives up, the kernel
+ * records PA_ERR_TIMEOUT in the device status word and exits normally; the
+ * CUDA context stays usable.  Used by tests of the failure path.
+ */
+int pa_selftest_timeout(int limit_us, void* stream);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_ATTN_H_ */

@@ -1,0 +1,136 @@
+"""The C ABI on the host: the library builds, loads, exports every symbol of
+include/pa_attn.h, and rejects bad arguments with the documented codes.
+
+Every call here returns before any CUDA API is touched (argument checks come
+first), so this file runs on a machine without a GPU.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from context_blocks_b200 import _binding as B
+from context_blocks_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_expected_api():
+    names = _declared_functions()
+    assert "pa_attn_fwd" in names and "pa_attn_merge" in names
+    assert names == sorted(B.SIGNATURES), (names, sorted(B.SIGNATURES))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_codes_match_header():
+    text = open(HEADER).read()
+    codes = {m.group(1): int(m.group(2)) for m in
+             re.finditer(r"#define\s+(PA_\w+)\s+\(?(-?\d+)\)?", text)}
+    for name in ("PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_MISALIGNED",
+                 "PA_ERR_CUDA", "PA_ERR_TIMEOUT"):
+        assert codes[name] == getattr(B, name), name
+
+
+def test_status_strings(lib):
+    assert B.status_string(0) == "PA_OK"
+    for code in (-1, -2, -3, -4, -5):
+        assert B.status_string(code).startswith("PA_ERR_")
+    assert B.status_string(12345) == "unknown status code"
+    assert B.version() == 100
+
+
+A = 1 << 20          # a 16-byte aligned fake address; never dereferenced
+MB = 1 << 24
+
+
+def _fwd(lib, q=A, k=A + MB, v=A + 2 * MB, o=A + 3 * MB, lse=A + 4 * MB, Bn=1, H=1, Nq=8, Nk=8,
+         d=128, scale=0.125):
+    return lib.pa_attn_fwd(q, k, v, o, lse, Bn, H, Nq, Nk, d, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), B.PA_ERR_INVALID_ARG), (dict(k=0), B.PA_ERR_INVALID_ARG),
+    (dict(v=0), B.PA_ERR_INVALID_ARG), (dict(o=0), B.PA_ERR_INVALID_ARG),
+    (dict(lse=0), B.PA_ERR_INVALID_ARG),
+    (dict(Bn=0), B.PA_ERR_INVALID_ARG), (dict(H=-1), B.PA_ERR_INVALID_ARG),
+    (dict(Nq=-1), B.PA_ERR_INVALID_ARG), (dict(Nk=0), B.PA_ERR_INVALID_ARG),
+    (dict(scale=0.0), B.PA_ERR_INVALID_ARG), (dict(scale=-1.0), B.PA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.PA_ERR_INVALID_ARG), (dict(scale=float("inf")), B.PA_ERR_INVALID_ARG),
+    (dict(d=96), B.PA_ERR_UNSUPPORTED), (dict(d=256), B.PA_ERR_UNSUPPORTED),
+    (dict(Bn=256, H=256), B.PA_ERR_UNSUPPORTED),
+    (dict(q=A + 8), B.PA_ERR_MISALIGNED), (dict(o=A + 3 * MB + 4), B.PA_ERR_MISALIGNED),
+    (dict(lse=A + 4 * MB + 2), B.PA_ERR_MISALIGNED),
+    (dict(o=A), B.PA_ERR_INVALID_ARG),                        # o aliases q
+    (dict(lse=A + MB + 64), B.PA_ERR_INVALID_ARG),            # lse inside k
+    (dict(lse=A + 3 * MB + 16), B.PA_ERR_INVALID_ARG),        # lse inside o
+])
+def test_fwd_argument_checks(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+    assert B.last_error() != ""
+
+
+def test_fwd_empty_query_is_noop(lib):
+    assert _fwd(lib, Nq=0) == B.PA_OK
+
+
+def _merge(lib, op=A, lp=A + 8 * MB, n=2, o=A + 12 * MB, lse=A + 14 * MB, Bn=1, H=2, N=16, d=64):
+    return lib.pa_attn_merge(op, lp, n, o, lse, Bn, H, N, d, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(op=0), B.PA_ERR_INVALID_ARG), (dict(lp=0), B.PA_ERR_INVALID_ARG),
+    (dict(o=0), B.PA_ERR_INVALID_ARG), (dict(lse=0), B.PA_ERR_INVALID_ARG),
+    (dict(n=0), B.PA_ERR_INVALID_ARG), (dict(Bn=0), B.PA_ERR_INVALID_ARG),
+    (dict(N=-3), B.PA_ERR_INVALID_ARG), (dict(d=32), B.PA_ERR_UNSUPPORTED),
+    (dict(op=A + 4), B.PA_ERR_MISALIGNED), (dict(lse=A + 14 * MB + 1), B.PA_ERR_MISALIGNED),
+    (dict(o=A + 64), B.PA_ERR_INVALID_ARG),                   # o inside o_parts
+])
+def test_merge_argument_checks(lib, kw, code):
+    assert _merge(lib, **kw) == code
+
+
+def test_merge_empty_is_noop(lib):
+    assert _merge(lib, N=0) == B.PA_OK
+
+
+def test_selftest_limit_checked_first(lib):
+    assert lib.pa_selftest_timeout(0, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_selftest_timeout(2_000_000, None) == B.PA_ERR_INVALID_ARG
+
+
+def test_python_binding_type_checks():
+    import torch
+    q = torch.zeros((1, 1, 4, 64), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        B.attn_fwd(q, q, q)
+    qb = q.to(torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.attn_fwd(qb, qb, qb)          # host tensors are refused before the library
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="missing"):
+        B.load_library(str(tmp_path / "nope.so"))
+
+
+def test_build_flags_target_sm100a():
+    assert "arch=compute_100a,code=sm_100a" in build_mod.NVCC_FLAGS
