@@ -80,7 +80,7 @@ class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML (read only)
     from a thread while the timed region runs."""
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, torch_device: int, period_s: float = 0.02):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
@@ -89,9 +89,12 @@ class ClockSampler:
         self._nvml = None
         try:
             import pynvml
+            import torch
             pynvml.nvmlInit()
+            # NVML counts physical GPUs; match torch's device by UUID.
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
             self._nvml = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception as e:  # pragma: no cover - no NVML here
             self.error = str(e)
@@ -431,8 +434,7 @@ def run_ours(args):
 
     w = workloads.get(args.workload)
     peaks = _peaks()
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else local)
+    sampler = ClockSampler(local)
     res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier)
     if res["status"] != 0:
         raise SystemExit(f"device status {res['status']} after the timed region")

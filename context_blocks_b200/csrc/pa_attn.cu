@@ -159,7 +159,15 @@ int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, voi
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!st->fwd_attr[slot]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
+      // The kernel re-allocates registers between warpgroups with setmaxnreg;
+      // the split is only valid for the per-thread count it was designed for.
+      cudaFuncAttributes fa;
+      cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      if (fa.numRegs != pa::kLaunchRegs)
+        return fail(PA_ERR_UNSUPPORTED, "attn_fwd built with %d registers per thread, expected %d",
+                    fa.numRegs, pa::kLaunchRegs);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       st->fwd_attr[slot] = true;
     }
