@@ -335,7 +335,7 @@ def oracle_sample(w, seconds: float, seed_rows: int = 0):
     rows, description)."""
     import numpy as np
     import oracle
-    q, k, v = workloads.make_case(w, device="cpu", nq=min(w.Nq, 64))
+    q, k, v = workloads.make_case(w, device="cpu", nq=min(w.Nq, 4096))
     qn = q.double().numpy()
     kn, vn = k.double().numpy(), v.double().numpy()
 
@@ -348,10 +348,18 @@ def oracle_sample(w, seconds: float, seed_rows: int = 0):
             oracle.chunked_attention(qq, kn, vn, w.scale, w.chunks)
         return time.perf_counter() - t0
 
-    cal_rows = 8
-    t_cal = max(run(cal_rows), 1e-4)
-    rows = int(max(1, min(w.Nq, cal_rows * seconds / t_cal)))
+    # Two calibration passes: a short one, then one of about a tenth of the
+    # budget, so per-call overhead does not skew the row count.
+    rows = min(w.Nq, 8)
+    for frac in (0.01, 0.1):
+        t_cal = max(run(rows), 1e-4)
+        rows = int(max(1, min(w.Nq, rows * frac * seconds / t_cal)))
+    t_cal = max(run(rows), 1e-4)
+    rows = int(max(1, min(w.Nq, rows * seconds / t_cal)))
     t = run(rows)
+    while t < 0.6 * seconds and rows < w.Nq:     # time is not quite linear in rows
+        rows = int(min(w.Nq, rows * seconds / max(t, 1e-4)))
+        t = run(rows)
     fl = workloads.flops(w.B, w.H, rows, w.Nk, w.d)
     desc = (f"{w.name}: all {w.B}x{w.H} (batch x head) of {rows} query rows x {w.Nk} keys"
             f"{' in ' + str(len(w.chunks)) + ' chunks + merge' if len(w.chunks) > 1 else ''}, fp64 NumPy")

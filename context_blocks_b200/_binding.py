@@ -29,6 +29,7 @@ PA_ERR_TIMEOUT = -5
 _VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "pa_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
+    "pa_attn_fwd_pair": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _VP]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
     "pa_last_error": (ctypes.c_char_p, []),
@@ -108,11 +109,12 @@ def _check_bf16(name, t, ndim):
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
 
 
-def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=None):
+def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=None, pair: bool = False):
     """Attention of q [B,H,Nq,d] against one K/V chunk k, v [B,H,Nk,d].
 
     Returns (o [B,H,Nq,d] bf16, lse [B,H,Nq] fp32, natural log), written into
-    ``out`` / ``lse`` when given.  ``scale`` defaults to 1/sqrt(d).
+    ``out`` / ``lse`` when given.  ``scale`` defaults to 1/sqrt(d).  With
+    ``pair=True`` the CTA-pair kernel (``pa_attn_fwd_pair``, d = 128) runs.
     """
     import torch
     _check_bf16("q", q, 4)
@@ -134,10 +136,11 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
     elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 [B,H,Nq] tensor")
-    rc = load_library().pa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                    lse.data_ptr(), B, H, Nq, Nk, d, float(scale),
-                                    _stream_handle(stream, q.device))
-    _check(rc, "pa_attn_fwd")
+    lib = load_library()
+    fn = lib.pa_attn_fwd_pair if pair else lib.pa_attn_fwd
+    rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
+            float(scale), _stream_handle(stream, q.device))
+    _check(rc, "pa_attn_fwd_pair" if pair else "pa_attn_fwd")
     return out, lse
 
 

@@ -196,7 +196,7 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
 // Share of exponentials computed on the FMA pipe (see exp2_poly_x2): one pair
 // in kEmuEvery; 0 = all on MUFU.
 #ifndef PA_EMU_EVERY
-#define PA_EMU_EVERY 4
+#define PA_EMU_EVERY 0
 #endif
 constexpr int kEmuEvery = PA_EMU_EVERY;  // 0: every exponential on MUFU
 

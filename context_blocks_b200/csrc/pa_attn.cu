@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "attn_fwd.cuh"
+#include "attn_fwd_pair.cuh"
 #include "lse_merge.cuh"
 #include "pa_attn.h"
 
@@ -59,7 +60,9 @@ struct DeviceState {
   int sm_count = 0;
   int* status = nullptr;  // device address of pa::g_status
   bool fwd_attr[2] = {false, false};
+  bool pair_attr = false;
 };
+
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -127,16 +130,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 3-D map over a [BH, N, d] bf16 tensor: box of 64 head-dim elements x 128
-// rows x 1, 128-byte swizzle, zero fill outside the tensor.
-int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh) {
+// 3-D map over a [BH, N, d] bf16 tensor: box of 64 head-dim elements x
+// box_rows rows x 1, 128-byte swizzle, zero fill outside the tensor.
+int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n_rows),
                         static_cast<cuuint64_t>(bh)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(n_rows) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(pa::kBM), 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -151,9 +154,9 @@ int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, voi
   using L = pa::FwdLayout<D>;
   CUtensorMap tq, tk, tv;
   int rc;
-  if ((rc = encode_map(&tq, q, D, Nq, BH)) != PA_OK) return rc;
-  if ((rc = encode_map(&tk, k, D, Nk, BH)) != PA_OK) return rc;
-  if ((rc = encode_map(&tv, v, D, Nk, BH)) != PA_OK) return rc;
+  if ((rc = encode_map(&tq, q, D, Nq, BH, pa::kBM)) != PA_OK) return rc;
+  if ((rc = encode_map(&tk, k, D, Nk, BH, pa::kBN)) != PA_OK) return rc;
+  if ((rc = encode_map(&tv, v, D, Nk, BH, pa::kBN)) != PA_OK) return rc;
   auto kern = pa::attn_fwd_kernel<D>;
   const int slot = (D == 64) ? 0 : 1;
   {
@@ -188,6 +191,61 @@ int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, voi
   return PA_OK;
 }
 
+// CTA-pair forward (head dim 128): clusters of two CTAs, 512 query rows each.
+int launch_fwd_pair(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int BH,
+                    int Nq, int Nk, float scale, cudaStream_t stream) {
+  using L = pa::PairLayout;
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = encode_map(&tq, q, 128, Nq, BH, pa::kBM)) != PA_OK) return rc;
+  if ((rc = encode_map(&tk, k, 128, Nk, BH, pa::kBN / 2)) != PA_OK) return rc;
+  if ((rc = encode_map(&tv, v, 128, Nk, BH, pa::kBN)) != PA_OK) return rc;
+  auto kern = pa::attn_fwd_pair_kernel<128>;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!st->pair_attr) {
+      // The kernel re-allocates registers between warpgroups with setmaxnreg;
+      // the split is only valid for the per-thread count it was designed for.
+      cudaFuncAttributes fa;
+      cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      if (fa.numRegs != pa::kLaunchRegs)
+        return fail(PA_ERR_UNSUPPORTED, "attn_fwd_pair built with %d registers per thread, expected %d",
+                    fa.numRegs, pa::kLaunchRegs);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      st->pair_attr = true;
+    }
+  }
+  pa::FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.n_kv_tiles = (Nk + pa::kBN - 1) / pa::kBN;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.status = st->status;
+  prm.timeout_ns = kDefaultTimeoutNs;
+  const int rows_per_pair = 2 * pa::kQTiles * pa::kBM;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ((Nq + rows_per_pair - 1) / rows_per_pair), BH);
+  cfg.blockDim = dim3(pa::kFwdThreads);
+  cfg.dynamicSmemBytes = L::kAllocBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, prm);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_pair launch");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_pair launch");
+  return PA_OK;
+}
+
 template <int D>
 int launch_merge(DeviceState* st, const void* o_parts, const float* lse_parts, int n_parts, void* o,
                  float* lse, long long rows, cudaStream_t stream) {
@@ -205,11 +263,13 @@ int launch_merge(DeviceState* st, const void* o_parts, const float* lse_parts, i
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
-                int Nk, int d, float scale, void* stream) {
-  g_err[0] = '\0';
+// Argument checks shared by the forward entry points.  On PA_OK, *st is the
+// current device's state, or null when there is nothing to do (Nq == 0).
+int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                   int d, float scale, DeviceState** st) {
+  *st = nullptr;
   if (!q || !k || !v || !o || !lse) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
   if (B < 1 || H < 1) return fail(PA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
   if (Nq < 0) return fail(PA_ERR_INVALID_ARG, "Nq must be >= 0 (got %d)", Nq);
@@ -238,11 +298,32 @@ int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   const char* names[5] = {"q", "k", "v", "o", "lse"};
   for (int i = 0; i < 5; ++i)
     if ((rc = check_device_ptr(ptrs[i], names[i], &dev)) != PA_OK) return rc;
+  return device_state(dev, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                int Nk, int d, float scale, void* stream) {
+  g_err[0] = '\0';
   DeviceState* st = nullptr;
-  if ((rc = device_state(dev, &st)) != PA_OK) return rc;
+  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st);
+  if (rc != PA_OK || st == nullptr) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_fwd<64>(st, q, k, v, o, lse, static_cast<int>(bh), Nq, Nk, scale, s);
-  return launch_fwd<128>(st, q, k, v, o, lse, static_cast<int>(bh), Nq, Nk, scale, s);
+  if (d == 64) return launch_fwd<64>(st, q, k, v, o, lse, B * H, Nq, Nk, scale, s);
+  return launch_fwd<128>(st, q, k, v, o, lse, B * H, Nq, Nk, scale, s);
+}
+
+int pa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                     int Nk, int d, float scale, void* stream) {
+  g_err[0] = '\0';
+  DeviceState* st = nullptr;
+  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st);
+  if (rc != PA_OK || st == nullptr) return rc;
+  if (d != 128) return fail(PA_ERR_UNSUPPORTED, "d must be 128 for the CTA-pair kernel (got %d)", d);
+  return launch_fwd_pair(st, q, k, v, o, lse, B * H, Nq, Nk, scale, static_cast<cudaStream_t>(stream));
 }
 
 int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void* o, float* lse, int B, int H,

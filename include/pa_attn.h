@@ -82,6 +82,20 @@ int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
                 int Nq, int Nk, int d, float scale, void* stream);
 
 /*
+ * pa_attn_fwd_pair - pa_attn_fwd computed on pairs of CTAs.
+ *
+ * Same operation, arguments, layouts, ownership and errors as pa_attn_fwd
+ * (diffusers "Context parallelism", section "Ring Attention"), for d = 128
+ * only (PA_ERR_UNSUPPORTED otherwise).  Two CTAs of a thread-block cluster
+ * share each tensor-core MMA (tcgen05 cta_group::2, M = 256), so each CTA
+ * loads only half of every K and V tile.  Results agree with pa_attn_fwd
+ * within rounding; which of the two is faster depends on the shape (the
+ * benchmark reports both).
+ */
+int pa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                     int Nq, int Nk, int d, float scale, void* stream);
+
+/*
  * pa_attn_merge - combine n partial results over disjoint key chunks.
  *
  * For every row r of the B*H*N rows (same section as above: the per-block

@@ -134,3 +134,11 @@ def test_missing_library_fails_loudly(tmp_path):
 
 def test_build_flags_target_sm100a():
     assert "arch=compute_100a,code=sm_100a" in build_mod.NVCC_FLAGS
+
+
+def test_pair_argument_checks(lib):
+    f = lib.pa_attn_fwd_pair
+    assert f(0, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 128, 0.1, None) == B.PA_ERR_INVALID_ARG
+    assert f(A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 96, 0.1, None) == B.PA_ERR_UNSUPPORTED
+    assert f(A + 8, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 128, 0.1, None) == B.PA_ERR_MISALIGNED
+    assert f(A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 0, 8, 128, 0.1, None) == B.PA_OK

@@ -309,3 +309,60 @@ def test_bounded_wait_times_out_and_reports(pa):
     o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), w.scale)
     assert_close(o, lse, o_ref, l_ref, "after timeout self-test")
     assert pa.poll_device_status() == pa.PA_OK
+
+
+# ---------------------------------------------------------------- CTA-pair kernel
+
+def _pair_case(pa, q, k, v, scale, what):
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:3], float("nan"), device="cuda")
+    pa.attn_fwd(q, k, v, scale=scale, out=o, lse=lse, pair=True)
+    torch.cuda.synchronize()
+    assert pa.poll_device_status() == pa.PA_OK
+    o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), scale)
+    assert_close(o, lse, o_ref, l_ref, what)
+    return o, lse
+
+
+def test_pair_flux(pa):
+    w = workloads.get("flux")
+    q, k, v = workloads.make_case(w, device="cuda")
+    o, lse = _pair_case(pa, q, k, v, w.scale, "pair flux")
+    o1, l1 = pa.attn_fwd(q, k, v, scale=w.scale)
+    torch.cuda.synchronize()
+    # the two kernels compute the same values in the same order per row
+    assert (o.float() - o1.float()).abs().max().item() <= 2 ** -8
+    assert (lse - l1).abs().max().item() <= 1e-5
+
+
+def test_pair_uneven_tail_chunk(pa):
+    w = workloads.get("tails")
+    q, k, v = workloads.make_case(w, device="cuda")
+    _pair_case(pa, q, k[:, :, :1151].contiguous(), v[:, :, :1151].contiguous(), w.scale, "pair tails chunk")
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d", [e for e in EDGE if e[4] == 128])
+def test_pair_edge_shapes(pa, B, H, Nq, Nk, d):
+    g = torch.Generator(device="cuda").manual_seed(2000 + Nq * 7 + Nk * 13)
+    q = torch.randn((B, H, Nq, d), generator=g, device="cuda").to(torch.bfloat16)
+    k = torch.randn((B, H, Nk, d), generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn((B, H, Nk, d), generator=g, device="cuda").to(torch.bfloat16)
+    _pair_case(pa, q, k, v, 1.0 / math.sqrt(d), f"pair edge {(B, H, Nq, Nk, d)}")
+
+
+def test_pair_rescale_path(pa):
+    B, H, Nq, Nk, d = 1, 2, 600, 1100, 128
+    g = torch.Generator(device="cuda").manual_seed(81)
+    q = torch.randn((B, H, Nq, d), generator=g, device="cuda") * 0.2 + 1.0
+    ramp = torch.linspace(0.0, 1.0, Nk, device="cuda")[None, None, :, None]
+    k = torch.randn((B, H, Nk, d), generator=g, device="cuda") * 0.1 + ramp * 6.0
+    v = torch.randn((B, H, Nk, d), generator=g, device="cuda")
+    q, k, v = (x.to(torch.bfloat16).contiguous() for x in (q, k, v))
+    _pair_case(pa, q, k, v, 1.0 / math.sqrt(d), "pair rising logits")
+
+
+def test_pair_rejects_head_dim_64(pa):
+    q = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(pa.PaError) as e:
+        pa.attn_fwd(q, q.clone(), q.clone(), pair=True)
+    assert e.value.code == pa.PA_ERR_UNSUPPORTED
