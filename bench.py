@@ -166,9 +166,10 @@ def aggregate_throughput(flops_per_step_per_rank: float, steps: int, world: int,
 class Step:
     """Buffers and launches of one hot-path step on one workload."""
 
-    def __init__(self, w: workloads.Workload, sets: int, device):
+    def __init__(self, w: workloads.Workload, sets: int, device, pair: bool = False):
         import torch
         self.w = w
+        self.pair = pair
         self.sets = []
         n = len(w.chunks)
         for s in range(sets):
@@ -200,7 +201,7 @@ class Step:
             ls = lse if n == 1 else lse_parts[p]
             if fwd_events is not None:
                 fwd_events[0].append(_record())
-            pa.attn_fwd(q, k, v, scale=self.w.scale, out=out, lse=ls)
+            pa.attn_fwd(q, k, v, scale=self.w.scale, out=out, lse=ls, pair=self.pair)
             if fwd_events is not None:
                 fwd_events[1].append(_record())
         if n > 1:
@@ -223,11 +224,11 @@ def _sets_for(w: workloads.Workload) -> int:
     return max(1, min(8, math.ceil(2.5 * L2_BYTES / per_set)))
 
 
-def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None):
+def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, pair=False):
     """Device time of `steps` steps (CUDA events on the launching stream,
     synchronised on both sides).  Returns a dict of timings."""
     import torch
-    st = Step(w, _sets_for(w), device)
+    st = Step(w, _sets_for(w), device, pair=pair)
     for i in range(warmup):
         st.run(i, pa)
     torch.cuda.synchronize()
@@ -516,6 +517,12 @@ def extra_measurements(pa, device, peaks):
             ent["merge_gbs"] = mb / (ent["merge_ms"] * 1e-3) / 1e9
         ent["pct_of_bf16_peak"] = 100.0 * ent["fwd_tflops"] / peaks["bf16_tflops"]
         out[name] = ent
+    # The CTA-pair forward kernel (pa_attn_fwd_pair) on the FLUX-shaped workload.
+    wf = workloads.get("flux")
+    r = time_workload(pa, wf, 200, 10, device, pair=True)
+    fl = workloads.flops(wf.B, wf.H, wf.Nq, wf.Nk, wf.d)
+    out["flux_pair_kernel"] = {"fwd_ms_per_launch": statistics.fmean(r["fwd_ms"]),
+                               "fwd_tflops": fl / (statistics.fmean(r["fwd_ms"]) * 1e-3) / 1e12}
     w8 = workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8)
     r = time_workload(pa, w8, 2, 1, device)
     fl = workloads.flops(w8.B, w8.H, w8.Nq, w8.Nk, w8.d)
