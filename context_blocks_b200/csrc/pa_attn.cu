@@ -20,6 +20,13 @@ namespace pa {
 // Device status word: kernels record the first device-side error here.
 __device__ int g_status = 0;
 
+// Scratch for pa_attn_chunks_noalloc: the per-chunk partial outputs and LSEs
+// live here instead of in memory the caller or the library allocates.  Every
+// GPU that loads the library holds these 32 MiB until the process exits.
+constexpr unsigned long long kNoAllocScratchBytes = 32ull << 20;
+constexpr int kNoAllocMaxChunks = 64;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 __global__ void timeout_probe_kernel(unsigned long long limit_ns, int* status) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_word;
@@ -59,6 +66,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int* status = nullptr;  // device address of pa::g_status
+  unsigned char* noalloc_scratch = nullptr;  // device address of pa::g_noalloc_scratch
   bool fwd_attr[2] = {false, false};
   bool pair_attr = false;
 };
@@ -85,6 +93,12 @@ int device_state(int dev, DeviceState** out) {
       e = cudaGetSymbolAddress(&addr, pa::g_status);
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
       s.status = static_cast<int*>(addr);
+      // In host code the array's name is only a host-side stand-in: the
+      // kernels must be given this device address instead.
+      void* scratch = nullptr;
+      e = cudaGetSymbolAddress(&scratch, pa::g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+      s.noalloc_scratch = static_cast<unsigned char*>(scratch);
     }
     s.ready = true;
   }
@@ -358,6 +372,49 @@ int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64) return launch_merge<64>(st, o_parts, lse_parts, n_parts, o, lse, rows, s);
   return launch_merge<128>(st, o_parts, lse_parts, n_parts, o, lse, rows, s);
+}
+
+int pa_attn_chunks_noalloc(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+                           const int* nk_chunks, int n_chunks, void* o, float* lse, int B, int H, int Nq, int d,
+                           float scale, void* stream) {
+  g_err[0] = '\0';
+  if (!q || !k_chunks || !v_chunks || !nk_chunks || !o || !lse)
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (n_chunks < 1 || n_chunks > pa::kNoAllocMaxChunks)
+    return fail(PA_ERR_INVALID_ARG, "n_chunks must be in [1, %d] (got %d)", pa::kNoAllocMaxChunks, n_chunks);
+  if (B < 1 || H < 1 || Nq < 0) return fail(PA_ERR_INVALID_ARG, "B, H must be >= 1 and Nq >= 0");
+  if (d != 64 && d != 128) return fail(PA_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  // Partials: n blocks of [B*H, Nq, d] bf16, then n blocks of [B*H, Nq] fp32.
+  const unsigned long long rows = static_cast<unsigned long long>(B) * H * Nq;
+  const unsigned long long o_part = rows * d * 2;
+  const unsigned long long lse_off = ((o_part * n_chunks) + 255ull) & ~255ull;
+  const unsigned long long need = (n_chunks > 1) ? lse_off + rows * 4ull * n_chunks : 0ull;
+  if (need > pa::kNoAllocScratchBytes)
+    return fail(PA_ERR_INVALID_ARG, "the %d partial results need %llu bytes of scratch; the limit is %llu", n_chunks,
+                need, pa::kNoAllocScratchBytes);
+  DeviceState* st = nullptr;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int rc = check_fwd_args(q, k_chunks[c], v_chunks[c], o, lse, B, H, Nq, nk_chunks[c], d, scale, &st);
+    if (rc != PA_OK) return rc;
+  }
+  if (st == nullptr) return PA_OK;  // Nq == 0
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int bh = B * H;
+  auto fwd = [&](const void* k, const void* v, void* out, float* out_lse, int nk) {
+    return d == 64 ? launch_fwd<64>(st, q, k, v, out, out_lse, bh, Nq, nk, scale, s)
+                   : launch_fwd<128>(st, q, k, v, out, out_lse, bh, Nq, nk, scale, s);
+  };
+  if (n_chunks == 1) return fwd(k_chunks[0], v_chunks[0], o, lse, nk_chunks[0]);
+  // Every forward below writes its whole partial block before the merge reads
+  // it, so nothing left in the shared array by an earlier call is ever read.
+  unsigned char* scratch = st->noalloc_scratch;
+  float* lse_parts = reinterpret_cast<float*>(scratch + lse_off);
+  for (int c = 0; c < n_chunks; ++c) {
+    const int rc = fwd(k_chunks[c], v_chunks[c], scratch + o_part * c, lse_parts + rows * c, nk_chunks[c]);
+    if (rc != PA_OK) return rc;
+  }
+  return d == 64 ? launch_merge<64>(st, scratch, lse_parts, n_chunks, o, lse, static_cast<long long>(rows), s)
+                 : launch_merge<128>(st, scratch, lse_parts, n_chunks, o, lse, static_cast<long long>(rows), s);
 }
 
 const char* pa_status_string(int code) {

@@ -117,6 +117,41 @@ int pa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float
 int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void* o, float* lse,
                   int B, int H, int N, int d, void* stream);
 
+/*
+ * pa_attn_chunks_noalloc - attention of Q over several K/V chunks, allocating
+ * nothing.
+ *
+ * Not part of the method: the pages have no counterpart for this call.  It is
+ * for callers that cannot allocate device memory on the call path: code that
+ * runs under a framework's caching allocator with a fixed memory budget,
+ * loops where cudaMalloc's implicit device-wide synchronisation is not
+ * acceptable, or plug-ins that are handed only their input and output
+ * buffers.  It gives the same result as pa_attn_fwd on each chunk into
+ * caller-allocated partial buffers followed by pa_attn_merge, but keeps the
+ * partials in a fixed 32 MiB array that the library reserves statically on
+ * every GPU that loads it (for as long as the process lives).
+ *
+ * q            [B,H,Nq,d] bf16, device, 16-byte aligned               (input)
+ * k_chunks[c], v_chunks[c]  [B,H,nk_chunks[c],d] bf16, device,
+ *              16-byte aligned, c < n_chunks; the three arrays are HOST arrays
+ * o, lse       as pa_attn_fwd                                         (output)
+ * n_chunks     1 .. 64; with n_chunks >= 2 the partials need
+ *              round_up(n*B*H*Nq*d*2, 256) + n*B*H*Nq*4 bytes, at most 32 MiB
+ *              (PA_ERR_INVALID_ARG beyond it, before anything is enqueued)
+ * B, H, Nq, d, scale, stream   as pa_attn_fwd; nk_chunks[c] >= 1
+ *
+ * Calls no allocating routine of any kind.  The first call on a device looks
+ * up the array's device address (once per device, with that device current);
+ * make that first call before any stream capture.  All calls on a device share
+ * the one array: calls whose work overlaps on the GPU (different streams, or
+ * other host threads) race on it and must be serialised by the caller.  The
+ * array keeps the last call's contents; each call writes every partial it
+ * reads, so nothing needs clearing.  Errors as pa_attn_fwd.
+ */
+int pa_attn_chunks_noalloc(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+                           const int* nk_chunks, int n_chunks, void* o, float* lse, int B, int H, int Nq,
+                           int d, float scale, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* pa_status_string(int code);
 
