@@ -50,7 +50,7 @@ NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "capture": None}
 
 def _kernel_digest() -> str:
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "attn_fwd.cuh"):
+    for f in ("ptx.cuh", "fwd_common.cuh", "attn_fwd.cuh"):
         with open(os.path.join(ROOT, "context_blocks_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()

@@ -24,9 +24,52 @@
 // The loads are plain per-CTA loads: nothing in this kernel multicasts data.
 #pragma once
 
-#include "attn_fwd.cuh"
+#include "fwd_common.cuh"
 
 namespace pa {
+namespace pairk {
+
+constexpr int kFwdThreads = 384;   // 12 warps = 3 warpgroups
+constexpr int kMmaWarp = 8;        // MMA issue for query tile 0 (tile 1: warp kMmaWarp + 2)
+constexpr int kTmaWarp = 9;        // warp 11 only completes warpgroup 2
+// Registers: the kernel is launched with kLaunchRegs per thread (what ptxas
+// assigns under __launch_bounds__(384, 1); the host refuses to launch if it
+// differs).  Warpgroup 2 (MMA issue, TMA, idle) then gives registers back and
+// the two softmax warpgroups take them:
+//   128 * kOtherRegs + 256 * kSoftmaxRegs == 384 * kLaunchRegs  (= 64512),
+// and per SMSP (one warp of each warpgroup) 224 + 224 + 56 <= 512.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
+static_assert(128 * kOtherRegs + 256 * kSoftmaxRegs == kFwdThreads * kLaunchRegs,
+              "register split must use exactly the launch allocation");
+
+// Exponential phase of the two softmax warpgroups runs in turns (warpgroup 0
+// on tile j, then warpgroup 1 on tile j, then warpgroup 0 on tile j+1, ...):
+// each then has the SM's MUFU units alone, and the tensor cores work on the
+// other warpgroup's P.V and next S meanwhile.
+#ifndef PA_SEQ_EXP
+#define PA_SEQ_EXP 1
+#endif
+constexpr bool kSeqExp = PA_SEQ_EXP != 0;
+
+
+// Threads issuing tcgen05.mma: 2 = one per query tile (warps 8 and 10),
+// 1 = warp 8 serves both tiles.
+#ifndef PA_MMA_THREADS
+#define PA_MMA_THREADS 2
+#endif
+constexpr int kMmaThreads = PA_MMA_THREADS;
+static_assert(kMmaThreads == 1 || kMmaThreads == 2, "one or two MMA-issuing threads");
+
+
+// Share of exponentials computed on the FMA pipe (see exp2_poly_x2): one pair
+// in kEmuEvery; 0 = all on MUFU.
+#ifndef PA_EMU_EVERY
+#define PA_EMU_EVERY 0
+#endif
+constexpr int kEmuEvery = PA_EMU_EVERY;  // 0: every exponential on MUFU
+
 
 constexpr int kPairStages = 8;  // K/V ring slots of 16 KB (one K half or one V half)
 
@@ -447,4 +490,5 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
+}  // namespace pairk
 }  // namespace pa

@@ -7,7 +7,7 @@ over [-1/2, 1/2]; the fit is an iteratively re-weighted least-squares
 (Lawson) iteration on Chebyshev nodes.  2^n is applied by adding n to the
 float32 exponent field.
 
-The printed coefficients are pasted into attn_fwd.cuh (kExp2C0..3).  The
+The printed coefficients are pasted into fwd_common.cuh (kExp2C0..3).  The
 second figure simulates the kernel's float32 arithmetic (magic-number
 rounding, Horner steps, exponent add) and reports its max relative error
 against float64 exp2 over [-126, 8].

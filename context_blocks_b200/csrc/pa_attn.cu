@@ -12,6 +12,7 @@
 
 #include "attn_fwd.cuh"
 #include "attn_fwd_pair.cuh"
+#include "fwd_common.cuh"
 #include "lse_merge.cuh"
 #include "pa_attn.h"
 
@@ -165,26 +166,18 @@ int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int
 template <int D>
 int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int BH,
                int Nq, int Nk, float scale, cudaStream_t stream) {
-  using L = pa::FwdLayout<D>;
+  using L = pa::single::FwdLayout<D>;
   CUtensorMap tq, tk, tv;
   int rc;
   if ((rc = encode_map(&tq, q, D, Nq, BH, pa::kBM)) != PA_OK) return rc;
   if ((rc = encode_map(&tk, k, D, Nk, BH, pa::kBN)) != PA_OK) return rc;
   if ((rc = encode_map(&tv, v, D, Nk, BH, pa::kBN)) != PA_OK) return rc;
-  auto kern = pa::attn_fwd_kernel<D>;
+  auto kern = pa::single::attn_fwd_kernel<D>;
   const int slot = (D == 64) ? 0 : 1;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!st->fwd_attr[slot]) {
-      // The kernel re-allocates registers between warpgroups with setmaxnreg;
-      // the split is only valid for the per-thread count it was designed for.
-      cudaFuncAttributes fa;
-      cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-      if (fa.numRegs != pa::kLaunchRegs)
-        return fail(PA_ERR_UNSUPPORTED, "attn_fwd built with %d registers per thread, expected %d",
-                    fa.numRegs, pa::kLaunchRegs);
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       st->fwd_attr[slot] = true;
     }
@@ -199,7 +192,7 @@ int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, voi
   prm.status = st->status;
   prm.timeout_ns = kDefaultTimeoutNs;
   dim3 grid((Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM), BH);
-  kern<<<grid, pa::kFwdThreads, L::kAllocBytes, stream>>>(tq, tk, tv, prm);
+  kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, tk, tv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
   return PA_OK;
@@ -208,13 +201,13 @@ int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, voi
 // CTA-pair forward (head dim 128): clusters of two CTAs, 512 query rows each.
 int launch_fwd_pair(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int BH,
                     int Nq, int Nk, float scale, cudaStream_t stream) {
-  using L = pa::PairLayout;
+  using L = pa::pairk::PairLayout;
   CUtensorMap tq, tk, tv;
   int rc;
   if ((rc = encode_map(&tq, q, 128, Nq, BH, pa::kBM)) != PA_OK) return rc;
   if ((rc = encode_map(&tk, k, 128, Nk, BH, pa::kBN / 2)) != PA_OK) return rc;
   if ((rc = encode_map(&tv, v, 128, Nk, BH, pa::kBN)) != PA_OK) return rc;
-  auto kern = pa::attn_fwd_pair_kernel<128>;
+  auto kern = pa::pairk::attn_fwd_pair_kernel<128>;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!st->pair_attr) {
@@ -223,9 +216,9 @@ int launch_fwd_pair(DeviceState* st, const void* q, const void* k, const void* v
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kern);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-      if (fa.numRegs != pa::kLaunchRegs)
+      if (fa.numRegs != pa::pairk::kLaunchRegs)
         return fail(PA_ERR_UNSUPPORTED, "attn_fwd_pair built with %d registers per thread, expected %d",
-                    fa.numRegs, pa::kLaunchRegs);
+                    fa.numRegs, pa::pairk::kLaunchRegs);
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       st->pair_attr = true;
@@ -243,7 +236,7 @@ int launch_fwd_pair(DeviceState* st, const void* q, const void* k, const void* v
   const int rows_per_pair = 2 * pa::kQTiles * pa::kBM;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ((Nq + rows_per_pair - 1) / rows_per_pair), BH);
-  cfg.blockDim = dim3(pa::kFwdThreads);
+  cfg.blockDim = dim3(pa::pairk::kFwdThreads);
   cfg.dynamicSmemBytes = L::kAllocBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -1,7 +1,7 @@
 """The FMA-pipe exp2 used for a share of the softmax exponentials.
 
 The kernel computes 2^x = 2^n * p(f) with n = round(x), f = x - n and a
-degree-3 polynomial p (coefficients in attn_fwd.cuh, fitted by
+degree-3 polynomial p (coefficients in fwd_common.cuh, fitted by
 csrc/gen_exp2_poly.py).  Here the same float32 steps are simulated in NumPy
 and held against float64 exp2: the relative error must stay far below the
 bf16 rounding step (2^-9) that P is stored with.
@@ -20,7 +20,7 @@ import gen_exp2_poly  # noqa: E402
 
 
 def _kernel_coeffs():
-    text = open(os.path.join(CSRC, "attn_fwd.cuh")).read()
+    text = open(os.path.join(CSRC, "fwd_common.cuh")).read()
     vals = [float(re.search(rf"kExp2C{i}\s*=\s*([-0-9.eE+]+)f", text).group(1)) for i in range(4)]
     return np.array(vals, dtype=np.float32)
 
