@@ -39,6 +39,23 @@
 namespace pa {
 namespace single {
 
+// Softmax arithmetic variants, measured against each other (all compute the
+// same values up to rounding order):
+//   PA_SINGLE_MAX3    row max as 8 chains of 3-input max instead of one chain
+//   PA_SINGLE_F2      scale-and-subtract and row sum on packed f32x2 pairs,
+//                     row sum in 4 partial sums
+//   PA_SINGLE_EMU     one exponential pair in PA_SINGLE_EMU on the FMA pipe
+//                     (exp2_poly_x2), 0 = all on MUFU
+#ifndef PA_SINGLE_MAX3
+#define PA_SINGLE_MAX3 1
+#endif
+#ifndef PA_SINGLE_F2
+#define PA_SINGLE_F2 1
+#endif
+#ifndef PA_SINGLE_EMU
+#define PA_SINGLE_EMU 0
+#endif
+
 constexpr int kStages = 4;         // K/V ring slots (each holds one K or one V tile)
 constexpr int kFwdThreads = 320;   // 10 warps
 constexpr int kMmaWarp = 8;
@@ -274,14 +291,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
       for (int e = 0; e < kBN; ++e) s[e] = __uint_as_float(sr[e]);
       const int valid = p.Nk - j * kBN;  // keys of this tile inside the chunk
+      const bool full_tile = valid >= kBN;  // tail tiles keep every exponential on MUFU
       if (valid < kBN) {
 #pragma unroll
         for (int e = 0; e < kBN; ++e)
           if (e >= valid) s[e] = -INFINITY;
       }
+#if PA_SINGLE_MAX3
+      float m8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+      for (int e = 16; e < kBN; e += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = max3f(m8[k], s[e + k], s[e + 8 + k]);
+      float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], max3f(m8[5], m8[6], m8[7])));
+#else
       float mx = s[0];
 #pragma unroll
       for (int e = 1; e < kBN; ++e) mx = fmaxf(mx, s[e]);
+#endif
       mx *= c;
       float alpha = 1.f;
       bool rescale = false;
@@ -304,18 +333,50 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       const float neg_m = -m_ref;
+#if PA_SINGLE_F2
+      const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
+      uint64_t l4[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+#endif
 #pragma unroll
       for (int ch = 0; ch < kBN / 32; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(fmaf(s[ch * 32 + 2 * e], c, neg_m));
-          const float p1 = ex2_approx(fmaf(s[ch * 32 + 2 * e + 1], c, neg_m));
+          float p0, p1;
+#if PA_SINGLE_F2
+          const uint64_t x = f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2);
+          if (PA_SINGLE_EMU > 0 && full_tile && (e % (PA_SINGLE_EMU > 0 ? PA_SINGLE_EMU : 1)) == 0) {
+            f2_split(exp2_poly_x2(x), p0, p1);
+          } else {
+            float x0, x1;
+            f2_split(x, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          l4[e & 3] = f2_add(l4[e & 3], f2(p0, p1));
+#else
+          const float x0 = fmaf(s[ch * 32 + 2 * e], c, neg_m);
+          const float x1 = fmaf(s[ch * 32 + 2 * e + 1], c, neg_m);
+          if (PA_SINGLE_EMU > 0 && full_tile && (e % (PA_SINGLE_EMU > 0 ? PA_SINGLE_EMU : 1)) == 0) {
+            f2_split(exp2_poly_x2(f2(x0, x1)), p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
           l += p0 + p1;
+#endif
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st_x16(tS + ch * 16, pk);
       }
+#if PA_SINGLE_F2
+      {
+        const uint64_t t = f2_add(f2_add(l4[0], l4[1]), f2_add(l4[2], l4[3]));
+        float a, b;
+        f2_split(t, a, b);
+        l += a + b;
+      }
+#endif
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
