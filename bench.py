@@ -499,6 +499,29 @@ def run_ours(args):
     return 0
 
 
+def fused_timing(pa, w, steps, warmup, device):
+    """Device time of one pa_attn_fwd_chunks launch over the workload's chunks."""
+    import torch
+    q, k, v = workloads.make_case(w, device=device)
+    pairs = workloads.split_keys(k, v, w.chunks)
+    del k, v
+    kc, vc = [a for a, _ in pairs], [b for _, b in pairs]
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+    for _ in range(warmup):
+        pa.attn_fwd_chunks(q, kc, vc, scale=w.scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        pa.attn_fwd_chunks(q, kc, vc, scale=w.scale, out=o, lse=lse)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
+    return {"step_ms": ms, "tflops_step": fl / (ms * 1e-3) / 1e12, "launches_per_step": 1}
+
+
 def extra_measurements(pa, device, peaks):
     """Secondary lines: the other workloads' device throughput (not the
     headline value).  Bounded repetitions each."""
@@ -517,6 +540,12 @@ def extra_measurements(pa, device, peaks):
             ent["merge_gbs"] = mb / (ent["merge_ms"] * 1e-3) / 1e9
         ent["pct_of_bf16_peak"] = 100.0 * ent["fwd_tflops"] / peaks["bf16_tflops"]
         out[name] = ent
+    # The chunked workloads as one fused launch (pa_attn_fwd_chunks).
+    for name in ("ring", "tails"):
+        w = workloads.get(name)
+        out[name + "_fused"] = fused_timing(pa, w, steps=20, warmup=3, device=device)
+    out["hunyuan_8chunks_fused"] = fused_timing(
+        pa, workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8), steps=2, warmup=1, device=device)
     # The CTA-pair forward kernel (pa_attn_fwd_pair) on the FLUX-shaped workload.
     wf = workloads.get("flux")
     r = time_workload(pa, wf, 200, 10, device, pair=True)

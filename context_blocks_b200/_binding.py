@@ -30,6 +30,7 @@ _VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "pa_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_fwd_pair": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
+    "pa_attn_fwd_chunks": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _VP]),
     "pa_attn_chunks_noalloc": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
@@ -164,6 +165,41 @@ def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
                                       lse.data_ptr(), B, H, N, d,
                                       _stream_handle(stream, o_parts.device))
     _check(rc, "pa_attn_merge")
+    return out, lse
+
+
+def _chunk_arrays(q, k_chunks, v_chunks):
+    B, H, Nq, d = q.shape
+    n = len(k_chunks)
+    if n < 1 or len(v_chunks) != n:
+        raise ValueError("need at least one chunk and as many V chunks as K chunks")
+    for kc, vc in zip(k_chunks, v_chunks):
+        _check_bf16("k chunk", kc, 4)
+        _check_bf16("v chunk", vc, 4)
+        if kc.shape != vc.shape or kc.shape[:2] != (B, H) or kc.shape[3] != d:
+            raise ValueError("chunk shapes must be [B, H, n_c, d] matching q")
+    kp = (ctypes.c_void_p * n)(*[kc.data_ptr() for kc in k_chunks])
+    vp = (ctypes.c_void_p * n)(*[vc.data_ptr() for vc in v_chunks])
+    nk = (ctypes.c_int * n)(*[kc.shape[2] for kc in k_chunks])
+    return kp, vp, nk, n
+
+
+def attn_fwd_chunks(q, k_chunks, v_chunks, scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """Attention of q over the concatenation of the K/V chunks (up to 8) in a
+    single launch (``pa_attn_fwd_chunks``); no partial results are written."""
+    import torch
+    _check_bf16("q", q, 4)
+    B, H, Nq, d = q.shape
+    kp, vp, nk, n = _chunk_arrays(q, k_chunks, v_chunks)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    rc = load_library().pa_attn_fwd_chunks(q.data_ptr(), kp, vp, nk, n, out.data_ptr(), lse.data_ptr(),
+                                           B, H, Nq, d, float(scale), _stream_handle(stream, q.device))
+    _check(rc, "pa_attn_fwd_chunks")
     return out, lse
 
 

@@ -25,8 +25,8 @@ struct FwdParams {
   __nv_bfloat16* o;     // [B*H, Nq, D]
   float* lse;           // [B*H, Nq]
   int Nq;
-  int Nk;
-  int n_kv_tiles;       // ceil(Nk / kBN)
+  int Nk;               // keys in all chunks of the launch
+  int n_kv_tiles;       // key tiles in all chunks of the launch
   float scale_log2;     // scale * log2(e)
   int* status;          // device status word
   unsigned long long timeout_ns;

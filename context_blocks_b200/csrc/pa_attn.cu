@@ -163,15 +163,32 @@ int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int
   return PA_OK;
 }
 
+// Single-CTA forward over n_chunks K/V chunks (n_chunks = 1 for one chunk).
 template <int D>
-int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int BH,
-               int Nq, int Nk, float scale, cudaStream_t stream) {
+int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void* const* v, const int* nk,
+               int n_chunks, void* o, float* lse, int BH, int Nq, float scale, cudaStream_t stream) {
   using L = pa::single::FwdLayout<D>;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq;
+  pa::single::KvChunks kv;
   int rc;
   if ((rc = encode_map(&tq, q, D, Nq, BH, pa::kBM)) != PA_OK) return rc;
-  if ((rc = encode_map(&tk, k, D, Nk, BH, pa::kBN)) != PA_OK) return rc;
-  if ((rc = encode_map(&tv, v, D, Nk, BH, pa::kBN)) != PA_OK) return rc;
+  long long nk_total = 0, tiles_total = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    if ((rc = encode_map(&kv.k[c], k[c], D, nk[c], BH, pa::kBN)) != PA_OK) return rc;
+    if ((rc = encode_map(&kv.v[c], v[c], D, nk[c], BH, pa::kBN)) != PA_OK) return rc;
+    kv.nk[c] = nk[c];
+    kv.tiles[c] = (nk[c] + pa::kBN - 1) / pa::kBN;
+    kv.tile_start[c] = static_cast<int>(tiles_total);
+    nk_total += nk[c];
+    tiles_total += kv.tiles[c];
+  }
+  for (int c = n_chunks; c < pa::single::kMaxChunks; ++c) {
+    kv.nk[c] = 0;
+    kv.tiles[c] = 0;
+    kv.tile_start[c] = 0x7fffffff;  // never reached by a tile index
+  }
+  kv.n_chunks = n_chunks;
+  if (nk_total > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "more than 2^31 keys in one call");
   auto kern = pa::single::attn_fwd_kernel<D>;
   const int slot = (D == 64) ? 0 : 1;
   {
@@ -186,13 +203,13 @@ int launch_fwd(DeviceState* st, const void* q, const void* k, const void* v, voi
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.Nq = Nq;
-  prm.Nk = Nk;
-  prm.n_kv_tiles = (Nk + pa::kBN - 1) / pa::kBN;
+  prm.Nk = static_cast<int>(nk_total);
+  prm.n_kv_tiles = static_cast<int>(tiles_total);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.status = st->status;
   prm.timeout_ns = kDefaultTimeoutNs;
   dim3 grid((Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM), BH);
-  kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, tk, tv, prm);
+  kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, kv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
   return PA_OK;
@@ -275,7 +292,7 @@ namespace {
 // Argument checks shared by the forward entry points.  On PA_OK, *st is the
 // current device's state, or null when there is nothing to do (Nq == 0).
 int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
-                   int d, float scale, DeviceState** st) {
+                   int d, float scale, DeviceState** st, bool host_only = false) {
   *st = nullptr;
   if (!q || !k || !v || !o || !lse) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
   if (B < 1 || H < 1) return fail(PA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
@@ -298,6 +315,7 @@ int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* 
     if (overlap(ins[i], in_bytes[i], o, qbytes) || overlap(ins[i], in_bytes[i], lse, lbytes))
       return fail(PA_ERR_INVALID_ARG, "outputs overlap an input");
   if (overlap(o, qbytes, lse, lbytes)) return fail(PA_ERR_INVALID_ARG, "o and lse overlap");
+  if (host_only) return PA_OK;
 
   (void)cudaGetLastError();
   int dev = 0, rc;
@@ -319,8 +337,30 @@ int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st);
   if (rc != PA_OK || st == nullptr) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_fwd<64>(st, q, k, v, o, lse, B * H, Nq, Nk, scale, s);
-  return launch_fwd<128>(st, q, k, v, o, lse, B * H, Nq, Nk, scale, s);
+  if (d == 64) return launch_fwd<64>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, s);
+  return launch_fwd<128>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, s);
+}
+
+int pa_attn_fwd_chunks(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+                       const int* nk_chunks, int n_chunks, void* o, float* lse, int B, int H, int Nq, int d,
+                       float scale, void* stream) {
+  g_err[0] = '\0';
+  if (!q || !k_chunks || !v_chunks || !nk_chunks || !o || !lse)
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (n_chunks < 1 || n_chunks > pa::single::kMaxChunks)
+    return fail(PA_ERR_INVALID_ARG, "n_chunks must be in [1, %d] (got %d)", pa::single::kMaxChunks, n_chunks);
+  DeviceState* st = nullptr;
+  // Every chunk's host-side checks first, so no CUDA call is made for a bad table.
+  for (int pass = 0; pass < 2; ++pass)
+    for (int c = 0; c < n_chunks; ++c) {
+      const int rc = check_fwd_args(q, k_chunks[c], v_chunks[c], o, lse, B, H, Nq, nk_chunks[c], d, scale, &st,
+                                    pass == 0);
+      if (rc != PA_OK) return rc;
+    }
+  if (st == nullptr) return PA_OK;  // Nq == 0
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_fwd<64>(st, q, k_chunks, v_chunks, nk_chunks, n_chunks, o, lse, B * H, Nq, scale, s);
+  return launch_fwd<128>(st, q, k_chunks, v_chunks, nk_chunks, n_chunks, o, lse, B * H, Nq, scale, s);
 }
 
 int pa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
@@ -386,16 +426,19 @@ int pa_attn_chunks_noalloc(const void* q, const void* const* k_chunks, const voi
     return fail(PA_ERR_INVALID_ARG, "the %d partial results need %llu bytes of scratch; the limit is %llu", n_chunks,
                 need, pa::kNoAllocScratchBytes);
   DeviceState* st = nullptr;
-  for (int c = 0; c < n_chunks; ++c) {
-    const int rc = check_fwd_args(q, k_chunks[c], v_chunks[c], o, lse, B, H, Nq, nk_chunks[c], d, scale, &st);
-    if (rc != PA_OK) return rc;
-  }
+  // Every chunk's host-side checks first, so no CUDA call is made for a bad table.
+  for (int pass = 0; pass < 2; ++pass)
+    for (int c = 0; c < n_chunks; ++c) {
+      const int rc = check_fwd_args(q, k_chunks[c], v_chunks[c], o, lse, B, H, Nq, nk_chunks[c], d, scale, &st,
+                                    pass == 0);
+      if (rc != PA_OK) return rc;
+    }
   if (st == nullptr) return PA_OK;  // Nq == 0
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int bh = B * H;
   auto fwd = [&](const void* k, const void* v, void* out, float* out_lse, int nk) {
-    return d == 64 ? launch_fwd<64>(st, q, k, v, out, out_lse, bh, Nq, nk, scale, s)
-                   : launch_fwd<128>(st, q, k, v, out, out_lse, bh, Nq, nk, scale, s);
+    return d == 64 ? launch_fwd<64>(st, q, &k, &v, &nk, 1, out, out_lse, bh, Nq, scale, s)
+                   : launch_fwd<128>(st, q, &k, &v, &nk, 1, out, out_lse, bh, Nq, scale, s);
   };
   if (n_chunks == 1) return fwd(k_chunks[0], v_chunks[0], o, lse, nk_chunks[0]);
   // Every forward below writes its whole partial block before the merge reads

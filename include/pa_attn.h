@@ -82,6 +82,29 @@ int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
                 int Nq, int Nk, int d, float scale, void* stream);
 
 /*
+ * pa_attn_fwd_chunks - attention of Q over several K/V chunks in one launch.
+ *
+ * The local loop of Ring Attention fused (diffusers "Context parallelism",
+ * section "Ring Attention": attend to each block held, and after all blocks
+ * the result is the full-sequence attention): the keys are the concatenation
+ * of the chunks, in order, so o and lse are the exact attention over all of
+ * them, the same as pa_attn_fwd per chunk followed by pa_attn_merge, with no
+ * partial results written.  Chunks of unequal, ragged length are accepted
+ * (section "Ring Anything Attention": each block keeps its real length).
+ *
+ * q            [B,H,Nq,d] bf16, device, 16-byte aligned               (input)
+ * k_chunks[c], v_chunks[c]  [B,H,nk_chunks[c],d] bf16, device, 16-byte
+ *              aligned; the three arrays are HOST arrays of n_chunks entries
+ * n_chunks     1 .. 8; nk_chunks[c] >= 1
+ * o, lse, B, H, Nq, d, scale, stream   as pa_attn_fwd
+ *
+ * Errors: as pa_attn_fwd, for every chunk.
+ */
+int pa_attn_fwd_chunks(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+                       const int* nk_chunks, int n_chunks, void* o, float* lse, int B, int H, int Nq, int d,
+                       float scale, void* stream);
+
+/*
  * pa_attn_fwd_pair - pa_attn_fwd computed on pairs of CTAs.
  *
  * Same operation, arguments, layouts, ownership and errors as pa_attn_fwd

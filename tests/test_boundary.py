@@ -142,3 +142,25 @@ def test_pair_argument_checks(lib):
     assert f(A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 96, 0.1, None) == B.PA_ERR_UNSUPPORTED
     assert f(A + 8, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 128, 0.1, None) == B.PA_ERR_MISALIGNED
     assert f(A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 0, 8, 128, 0.1, None) == B.PA_OK
+
+
+def _chunks(lib, n=3, nk=(8, 8, 8), kaddr=None, Nq=8, d=128, q=A, o=A + 3 * MB, lse=A + 4 * MB):
+    kaddr = kaddr or [A + MB + c * 4096 for c in range(n)]
+    kp = (ctypes.c_void_p * max(n, 1))(*kaddr[:n])
+    vp = (ctypes.c_void_p * max(n, 1))(*[A + 2 * MB + c * 4096 for c in range(n)])
+    nkp = (ctypes.c_int * max(n, 1))(*nk[:n])
+    return lib.pa_attn_fwd_chunks(q, kp, vp, nkp, n, o, lse, 1, 1, Nq, d, 0.125, None)
+
+
+def test_fwd_chunks_argument_checks(lib):
+    assert lib.pa_attn_fwd_chunks(A, None, None, None, 1, A + 3 * MB, A + 4 * MB, 1, 1, 8, 128, 0.1,
+                                  None) == B.PA_ERR_INVALID_ARG
+    assert _chunks(lib, n=0) == B.PA_ERR_INVALID_ARG
+    assert _chunks(lib, n=9, nk=(8,) * 9, kaddr=[A + MB + c * 4096 for c in range(9)]) == B.PA_ERR_INVALID_ARG
+    assert "n_chunks" in B.last_error()
+    assert _chunks(lib, nk=(8, 0, 8)) == B.PA_ERR_INVALID_ARG          # an empty chunk
+    assert _chunks(lib, kaddr=[A + MB, A + MB + 4104, A + MB + 8192]) == B.PA_ERR_MISALIGNED
+    assert _chunks(lib, kaddr=[A + MB, 0, A + MB + 8192]) == B.PA_ERR_INVALID_ARG
+    assert _chunks(lib, d=96) == B.PA_ERR_UNSUPPORTED
+    assert _chunks(lib, o=A + MB + 4096) == B.PA_ERR_INVALID_ARG         # o overlaps a K chunk
+    assert _chunks(lib, Nq=0) == B.PA_OK                                 # empty query: nothing to do

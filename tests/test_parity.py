@@ -311,6 +311,73 @@ def test_bounded_wait_times_out_and_reports(pa):
     assert pa.poll_device_status() == pa.PA_OK
 
 
+# ---------------------------------------------------------------- fused chunks
+
+def _fused_check(pa, w, rows=None):
+    """pa_attn_fwd_chunks over the workload's chunks vs the oracle over all keys."""
+    q, k, v = workloads.make_case(w, device="cuda")
+    pairs = workloads.split_keys(k, v, w.chunks)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:3], float("nan"), device="cuda")
+    pa.attn_fwd_chunks(q, [a for a, _ in pairs], [b for _, b in pairs], scale=w.scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert pa.poll_device_status() == pa.PA_OK
+    qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
+    if rows is None:
+        o_ref, l_ref = oracle.attention(qh, kh, vh, w.scale)
+        assert_close(o, lse, o_ref, l_ref, f"fused chunks {w.name}")
+    else:
+        o_ref, l_ref = oracle.attention_rows(qh, kh, vh, w.scale, rows)
+        assert_close(o[:, :, rows], lse[:, :, rows], o_ref, l_ref, f"fused chunks {w.name} sampled rows")
+    return q, pairs, o, lse
+
+
+def test_fused_ring_step(pa):
+    w = workloads.get("ring")
+    q, pairs, o, lse = _fused_check(pa, w)
+    # same values as one forward per chunk followed by the merge
+    o2, l2 = pa.blockwise_attention(q, [a for a, _ in pairs], [b for _, b in pairs], scale=w.scale)
+    torch.cuda.synchronize()
+    # the per-chunk path rounds each partial O to bf16 before the merge; the
+    # fused launch rounds once, so the two differ by a few bf16 half-ulps at most
+    assert (o.float() - o2.float()).abs().max().item() <= 1e-2
+    assert (lse - l2).abs().max().item() <= 1e-3
+
+
+def test_fused_uneven_tails(pa):
+    _fused_check(pa, workloads.get("tails"))
+
+
+def test_fused_tiny_head_dim_64(pa):
+    _fused_check(pa, workloads.get("tiny"))
+
+
+def test_fused_ragged_and_single_key_chunks(pa):
+    w = workloads.Workload("ragged", B=1, H=2, Nq=300, Nk=260, d=128, rms_qk=False,
+                           chunks=(1, 128, 3, 127, 1), seed=31)
+    _fused_check(pa, w)
+
+
+def test_fused_eight_chunks_of_one_tile(pa):
+    w = workloads.Workload("eight", B=1, H=2, Nq=257, Nk=8 * 128, d=128, rms_qk=True,
+                           chunks=(128,) * 8, seed=32)
+    _fused_check(pa, w)
+
+
+@pytest.mark.slow
+def test_fused_hunyuan_eight_chunks(pa):
+    w = workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8)
+    _fused_check(pa, w, rows=_hunyuan_rows(w))
+
+
+def test_fused_rejects_more_than_eight_chunks(pa):
+    q = torch.zeros((1, 1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    ks = [torch.zeros((1, 1, 4, 128), dtype=torch.bfloat16, device="cuda") for _ in range(9)]
+    with pytest.raises(pa.PaError) as e:
+        pa.attn_fwd_chunks(q, ks, [x.clone() for x in ks])
+    assert e.value.code == pa.PA_ERR_INVALID_ARG
+
+
 # ---------------------------------------------------------------- CTA-pair kernel
 
 def _pair_case(pa, q, k, v, scale, what):
