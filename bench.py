@@ -45,7 +45,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attn_fwd launch on the default workload, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
 # kernel source whose digest is recorded with it.  See profiles/.
-NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "capture": None}
+NCU_TRAFFIC = {
+    "source_sha256": "78be64cc02328ba1230744048d229611863726660ed9f164ca1ce5daaeef77c0",
+    "bytes_per_launch": 84989952 + 5036288,   # dram__bytes_read.sum + dram__bytes_write.sum
+    "capture": "profiles/attn_fwd_flux.md",
+}
 
 
 def _kernel_digest() -> str:
@@ -457,7 +461,7 @@ def run_ours(args):
     fl_launch = fl / len(w.chunks)
     achieved = fl_launch / (fwd_mean_ms * 1e-3) / 1e12
     traffic = None
-    if NCU_TRAFFIC["source_sha256"] == _kernel_digest():
+    if w.name == "flux" and NCU_TRAFFIC["source_sha256"] == _kernel_digest():
         traffic = NCU_TRAFFIC["bytes_per_launch"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,

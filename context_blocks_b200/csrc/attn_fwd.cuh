@@ -55,52 +55,17 @@ namespace single {
 #ifndef PA_SINGLE_EMU
 #define PA_SINGLE_EMU 0
 #endif
+// Barrier waits:
+//   PA_WAIT_HINT      waits of the softmax warps and of the MMA-issuing thread
+//                     pass a long suspend-time hint to mbarrier.try_wait, so a
+//                     waiting thread sleeps until the phase completes instead
+//                     of probing the barrier again and again
+#ifndef PA_WAIT_HINT
+#define PA_WAIT_HINT 1
+#endif
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms; the wait itself stays bounded by the time limit
 
-//   PA_SINGLE_SPEC    exponentials of a tile with the previous reference max
-//                     while the tile max is taken; the tile is recomputed (S
-//                     reloaded from TMEM) only when the max moved past the
-//                     lazy-rescale threshold.  P is stored after the check.
-//   PA_MMA_SPIN       the MMA-issuing thread polls its barriers with
-//                     test_wait instead of suspending in try_wait
-//   PA_SINGLE_STAGES  K/V ring slots
-#ifndef PA_SINGLE_SPEC
-#define PA_SINGLE_SPEC 0
-#endif
-#ifndef PA_MMA_SPIN
-#define PA_MMA_SPIN 0
-#endif
-#ifndef PA_SINGLE_STAGES
-#define PA_SINGLE_STAGES 4
-#endif
-//   PA_MMA_ISSUERS    threads issuing tcgen05.mma: 1 = warp 8 serves both
-//                     query tiles; 2 = warp 8 serves tile 0 and warp 10 tile 1,
-//                     so one can issue while the other waits
-#ifndef PA_MMA_ISSUERS
-#define PA_MMA_ISSUERS 1
-#endif
-//   PA_MMA_WARP       the single issuer's loop runs on all 32 lanes of warp 8
-//                     (uniform control flow); lane 0 alone issues
-#ifndef PA_MMA_WARP
-#define PA_MMA_WARP 0
-#endif
-//   PA_SM_WAIT        softmax warps' wait for S: 0 = every lane polls with
-//                     try_wait, 1 = try_wait with a long suspend hint,
-//                     2 = lane 0 polls and the warp syncs on it
-//   PA_MMA_HINT       the MMA thread's waits use a long suspend hint
-//   PA_SINGLE_ROLL    the exponential loop rolled over 32-column chunks
-#ifndef PA_SINGLE_ROLL
-#define PA_SINGLE_ROLL 0
-#endif
-#ifndef PA_SM_WAIT
-#define PA_SM_WAIT 0
-#endif
-#ifndef PA_MMA_HINT
-#define PA_MMA_HINT 0
-#endif
-constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms: sleep until the phase completes
-static_assert(PA_MMA_ISSUERS == 1 || PA_MMA_ISSUERS == 2, "one or two MMA-issuing threads");
-
-constexpr int kStages = PA_SINGLE_STAGES;  // K/V ring slots (each holds one K or one V tile)
+constexpr int kStages = 4;         // K/V ring slots (each holds one K or one V tile)
 constexpr int kMaxChunks = 8;      // K/V chunks one launch can consume
 
 // The K/V chunks of one launch: keys are the concatenation of the chunks, in
@@ -115,11 +80,9 @@ struct KvChunks {
   int tile_start[kMaxChunks];  // key tiles before chunk c (unused entries: INT_MAX)
   int n_chunks;
 };
-constexpr int kIssuers = PA_MMA_ISSUERS;
-constexpr int kFwdThreads = 320 + 32 * (kIssuers - 1);   // 10 warps (11 with two issuers)
+constexpr int kFwdThreads = 320;   // 10 warps
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
-constexpr int kMmaWarp2 = 10;      // second issuer (query tile 1) when kIssuers == 2
 
 template <int D>
 struct FwdLayout {
@@ -130,8 +93,8 @@ struct FwdLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kQTiles * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain[2]
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 2;
+  // q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
   static constexpr int kBytes = kAbortOff + 4;
@@ -177,7 +140,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int i = 0; i < 2; ++i) mbar_init(bar_q_full0 + 8 * i, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar_kv_full0 + 8 * s, 1);
-      mbar_init(bar_kv_empty0 + 8 * s, kIssuers);  // one commit per issuing thread
+      mbar_init(bar_kv_empty0 + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_s_full0 + 8 * i, 1);
@@ -185,7 +148,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar_o_full0 + 8 * i, 1);
     }
     mbar_init(bar_drain, 1);
-    mbar_init(bar_drain + 8, 1);
     *abort_word = 0;
     fence_barrier_init();
   }
@@ -251,78 +213,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (kIssuers == 2 && (warp == kMmaWarp || warp == kMmaWarp2)) {
-    // ------------------------------------------------- MMA issue, one thread per query tile
-    if (lane == 0) {
-      const int i = (warp == kMmaWarp) ? 0 : 1;
-      constexpr uint32_t kIdS = idesc_bf16(128, kBN, false, false);
-      constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
-      const uint32_t tS = tmem + i * kBN;
-      const uint32_t tO = tmem + 2 * kBN + i * D;
-      const uint32_t sq = sQ + i * L::kTileBytes;
-      auto mma_wait = [&](uint32_t bar, uint32_t parity) {
-        return PA_MMA_SPIN ? mbar_wait_spin(bar, parity, abort_word, p.status, kStatusTimeout, lim)
-                           : mbar_wait(bar, parity, abort_word, p.status, kStatusTimeout, lim);
-      };
-      auto issue_qk = [&](uint32_t sK) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * L::kBoxBytes + (kk % 4) * 32;
-          umma_ss(tS, sdesc_k_sw128(sq + off), sdesc_k_sw128(sK + off), kIdS, kk > 0);
-        }
-      };
-      auto issue_pv = [&](uint32_t sV, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tO, tS + kk * 8, sdesc_mn_sw128(sV + kk * 2048, L::kBoxBytes), kIdPV, (acc || kk > 0) ? 1u : 0u);
-      };
-      bool ok = mma_wait(bar_q_full0 + 8 * i, 0) && mma_wait(bar_kv_full0, 0);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(sRing);
-        umma_commit(bar_s_full0 + 8 * i);
-        umma_commit(bar_kv_empty0);
-      }
-      int idx = 1;
-      for (int j = 0; j < n && ok; ++j) {
-        const int sv = idx % kStages;
-        const uint32_t uv = idx / kStages;
-        ++idx;
-        const bool more = (j + 1 < n);
-        const int sk = idx % kStages;
-        const uint32_t uk = idx / kStages;
-        if (more) ++idx;
-        if (!mma_wait(bar_kv_full0 + 8 * sv, uv & 1) || !mma_wait(bar_p_full0 + 8 * i, j & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        issue_pv(sRing + sv * L::kTileBytes, j > 0);
-        umma_commit(bar_kv_empty0 + 8 * sv);
-        if (more) {
-          if (!mma_wait(bar_kv_full0 + 8 * sk, uk & 1)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_qk(sRing + sk * L::kTileBytes);
-          umma_commit(bar_s_full0 + 8 * i);
-          umma_commit(bar_kv_empty0 + 8 * sk);
-        } else {
-          umma_commit(bar_o_full0 + 8 * i);
-        }
-      }
-      // Every MMA this thread issued completes before tensor memory is freed.
-      umma_commit(bar_drain + 8 * i);
-      mbar_wait(bar_drain + 8 * i, 0, nullptr, p.status, kStatusTimeout, lim);
-    }
-    __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
-    // With PA_MMA_WARP the whole warp runs this loop in step and lane 0
-    // alone issues; otherwise lane 0 runs it alone.
-    const uint32_t lead = (PA_MMA_WARP == 0 || lane == 0) ? 1u : 0u;
-    if (PA_MMA_WARP || lane == 0) {
+    if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, kBN, false, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
       const uint32_t tO0 = tmem + 2 * kBN;
@@ -333,7 +226,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * L::kBoxBytes + (kk % 4) * 32;
-          umma_ss_if(tmem + i * kBN, sdesc_k_sw128(sq + off), sdesc_k_sw128(sK + off), kIdS, kk > 0, lead);
+          umma_ss(tmem + i * kBN, sdesc_k_sw128(sq + off), sdesc_k_sw128(sK + off), kIdS, kk > 0);
         }
       };
       // O_i (+)= P_i V : P from TMEM (bf16 pairs, 8 columns per 16 keys),
@@ -341,14 +234,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       auto issue_pv = [&](int i, uint32_t sV, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts_if(tO0 + i * D, tmem + i * kBN + kk * 8, sdesc_mn_sw128(sV + kk * 2048, L::kBoxBytes),
-                     kIdPV, (acc || kk > 0) ? 1u : 0u, lead);
+          umma_ts(tO0 + i * D, tmem + i * kBN + kk * 8, sdesc_mn_sw128(sV + kk * 2048, L::kBoxBytes),
+                  kIdPV, (acc || kk > 0) ? 1u : 0u);
       };
 
       auto mma_wait = [&](uint32_t bar, uint32_t parity, volatile int* aw, int* st, int code, uint64_t limit) {
-        return PA_MMA_SPIN   ? mbar_wait_spin(bar, parity, aw, st, code, limit)
-               : PA_MMA_HINT ? mbar_wait_hint(bar, parity, aw, st, code, limit, kSuspendHintNs)
-                             : mbar_wait(bar, parity, aw, st, code, limit);
+        return PA_WAIT_HINT ? mbar_wait_hint(bar, parity, aw, st, code, limit, kSuspendHintNs)
+                            : mbar_wait(bar, parity, aw, st, code, limit);
       };
       bool ok = mbar_wait(bar_q_full0, 0, abort_word, p.status, kStatusTimeout, lim) &&
                 mbar_wait(bar_q_full0 + 8, 0, abort_word, p.status, kStatusTimeout, lim) &&
@@ -356,10 +248,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok) {
         tc_fence_after();
         issue_qk(0, sRing);
-        umma_commit_if(bar_s_full0, lead);
+        umma_commit(bar_s_full0);
         issue_qk(1, sRing);
-        umma_commit_if(bar_s_full0 + 8, lead);
-        umma_commit_if(bar_kv_empty0, lead);
+        umma_commit(bar_s_full0 + 8);
+        umma_commit(bar_kv_empty0);
       }
       int idx = 1;
       for (int j = 0; j < n && ok; ++j) {
@@ -385,7 +277,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           tc_fence_after();
           issue_pv(i, sRing + sv * L::kTileBytes, j > 0);
-          if (i == 1) umma_commit_if(bar_kv_empty0 + 8 * sv, lead);
+          if (i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
           if (more) {
             if (i == 0) {
               if (!mma_wait(bar_kv_full0 + 8 * sk, uk & 1, abort_word, p.status, kStatusTimeout, lim)) {
@@ -395,15 +287,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tc_fence_after();
             }
             issue_qk(i, sRing + sk * L::kTileBytes);
-            umma_commit_if(bar_s_full0 + 8 * i, lead);
-            if (i == 1) umma_commit_if(bar_kv_empty0 + 8 * sk, lead);
+            umma_commit(bar_s_full0 + 8 * i);
+            if (i == 1) umma_commit(bar_kv_empty0 + 8 * sk);
           } else {
-            umma_commit_if(bar_o_full0 + 8 * i, lead);
+            umma_commit(bar_o_full0 + 8 * i);
           }
         }
       }
       // Every MMA this thread issued completes before tensor memory is freed.
-      umma_commit_if(bar_drain, lead);
+      umma_commit(bar_drain);
       mbar_wait(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
     }
     __syncwarp();
@@ -426,16 +318,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
       for (int cc = 1; cc < kMaxChunks; ++cc) chunk += (j >= kv.tile_start[cc]) ? 1 : 0;
       const int valid = kv.nk[chunk] - (j - kv.tile_start[chunk]) * kBN;  // keys of this tile in its chunk
-      bool got;
-      if (PA_SM_WAIT == 1) {
-        got = mbar_wait_hint(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim, kSuspendHintNs);
-      } else if (PA_SM_WAIT == 2) {
-        got = true;
-        if (lane == 0) got = mbar_wait(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim);
-        __syncwarp();
-      } else {
-        got = mbar_wait(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim);
-      }
+      const bool got =
+          PA_WAIT_HINT
+              ? mbar_wait_hint(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim, kSuspendHintNs)
+              : mbar_wait(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim);
       if (__any_sync(0xffffffffu, !got)) {
         ok = false;
         break;
@@ -452,101 +338,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int e = 0; e < kBN; ++e)
           if (e >= valid) s[e] = -INFINITY;
       }
-#if PA_SINGLE_SPEC
-      uint32_t pk[kBN / 2];  // P of this tile as bf16 pairs, stored once the max is settled
-      uint64_t l4[4];
-      auto exp_pass = [&](float neg_m, bool track, float (&m8)[8]) {
-        const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) l4[q4] = f2(0.f, 0.f);
-#pragma unroll
-        for (int ch = 0; ch < kBN / 32; ++ch) {
-          if (track) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              m8[k] = max3f(m8[k], s[ch * 32 + k], s[ch * 32 + 8 + k]);
-              m8[k] = max3f(m8[k], s[ch * 32 + 16 + k], s[ch * 32 + 24 + k]);
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float p0, p1;
-            const uint64_t x = f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2);
-            if (PA_SINGLE_EMU > 0 && full_tile && (e % (PA_SINGLE_EMU > 0 ? PA_SINGLE_EMU : 1)) == 0) {
-              f2_split(exp2_poly_x2(x), p0, p1);
-            } else {
-              float x0, x1;
-              f2_split(x, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            l4[e & 3] = f2_add(l4[e & 3], f2(p0, p1));
-            pk[ch * 16 + e] = pack_bf16x2(p0, p1);
-          }
-        }
-      };
-      auto l4_sum = [&]() {
-        const uint64_t t2 = f2_add(f2_add(l4[0], l4[1]), f2_add(l4[2], l4[3]));
-        float a, b;
-        f2_split(t2, a, b);
-        return a + b;
-      };
-      auto max8 = [&](const float (&m8)[8]) {
-        return fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], max3f(m8[5], m8[6], m8[7])));
-      };
-      float m8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
-      float tl;
-      if (j > 0) {
-        // Speculative pass at the current reference max; the tile max comes
-        // with it.  Accepted unless the max moved past the threshold.
-        exp_pass(-m_ref, true, m8);
-        tl = l4_sum();
-        const float mx = max8(m8) * c;
-        const bool redo = mx > m_ref + kRescaleLog2;
-        if (__any_sync(0xffffffffu, redo)) {
-          float alpha = 1.f;
-          if (redo) {
-            alpha = ex2_approx(m_ref - mx);
-            l *= alpha;
-            m_ref = mx;
-          }
-          // PV of tile j-1 has completed (S_i(j) was issued after it).
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t orr[32];
-            tmem_ld_x32(tO + ch * 32, orr);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st_x32(tO + ch * 32, orr);
-          }
-          // S is still in TMEM (P has not been stored): reload and redo.
-          tmem_ld_x128(tS, sr);
-#pragma unroll
-          for (int e = 0; e < kBN; ++e) s[e] = (e < valid) ? __uint_as_float(sr[e]) : -INFINITY;
-          exp_pass(-m_ref, false, m8);
-          tl = l4_sum();
-        }
-      } else {
-#pragma unroll
-        for (int ch = 0; ch < kBN / 32; ++ch)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            m8[k] = max3f(m8[k], s[ch * 32 + k], s[ch * 32 + 8 + k]);
-            m8[k] = max3f(m8[k], s[ch * 32 + 16 + k], s[ch * 32 + 24 + k]);
-          }
-        m_ref = max8(m8) * c;  // first tile: l = 0 and O is not yet written
-        exp_pass(-m_ref, false, m8);
-        tl = l4_sum();
-      }
-      l += tl;
-      tmem_st_x64(tS, pk);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p_full0 + 8 * i);
-#else
 #if PA_SINGLE_MAX3
       float m8[8];
 #pragma unroll
@@ -586,40 +377,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #if PA_SINGLE_F2
       const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
       uint64_t l4[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-#endif
-#if PA_SINGLE_ROLL
-      static_assert(PA_SINGLE_F2, "the rolled exponential loop uses the f32x2 forms");
-      // Rolled over the four 32-column chunks (small code); each chunk's S is
-      // re-read from TMEM, which still holds it: P of chunk ch goes to columns
-      // [16ch, 16ch + 16), below every column a later chunk reads.
-#pragma unroll 1
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t r32[32];
-        tmem_ld_x32(tS + ch * 32, r32);
-        float sc[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sc[e] = __uint_as_float(r32[e]);
-        const int vrel = valid - ch * 32;
-        if (vrel < 32) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (e >= vrel) sc[e] = -INFINITY;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float p0, p1;
-          const uint64_t x = f2_fma(f2(sc[2 * e], sc[2 * e + 1]), c2, nm2);
-          float x0, x1;
-          f2_split(x, x0, x1);
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
-          l4[e & 3] = f2_add(l4[e & 3], f2(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        tmem_st_x16(tS + ch * 16, pk);
-      }
-      if (false)
 #endif
 #pragma unroll
       for (int ch = 0; ch < kBN / 32; ++ch) {
@@ -665,7 +422,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p_full0 + 8 * i);
-#endif
     }
 
     if (ok) {
