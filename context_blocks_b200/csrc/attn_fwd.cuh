@@ -14,8 +14,9 @@
 // Kernel structure (one CTA per 256 query rows of one (b, h)):
 //   warps 0-3  softmax warpgroup for query tile 0 (rows   0..127 of the block)
 //   warps 4-7  softmax warpgroup for query tile 1 (rows 128..255 of the block)
-//   warp  8    TMEM allocation + single-thread tcgen05.mma issue
-//   warp  9    single-thread TMA producer (Q once, then K_j / V_j ring)
+//   warp  8    TMEM allocation + tcgen05.mma issue (the whole warp runs the
+//              loop in step, one elected lane issues)
+//   warp  9    TMA producer (Q once, then the K_j / V_j ring; same scheme)
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128)        S_0 = Q_0 K_j^T   (P_0 is written back over it as bf16)
 //   [128,256)      S_1 = Q_1 K_j^T   (P_1 likewise)
@@ -169,7 +170,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop in step; the elected lane issues the loads.
+    const bool leader = elect_one();
+    if (leader) {
       for (int i = 0; i < kQTiles; ++i) {
         mbar_arrive_expect_tx(bar_q_full0 + 8 * i, L::kTileBytes);
 #pragma unroll
@@ -177,127 +180,149 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tma_load_3d(sQ + i * L::kTileBytes + b * L::kBoxBytes, &tm_q, bar_q_full0 + 8 * i, b * 64,
                       q0 + i * kBM, bh);
       }
-      bool ok = true;
-      int idx = 0;  // ring loads issued so far
-      for (int jt = 0; jt < n && ok; ++jt) {
-        // Chunk of key tile jt and the tile's row offset inside that chunk.
-        int c = 0;
+    }
+    __syncwarp();
+    bool ok = true;
+    int idx = 0;  // ring loads issued so far
+    for (int jt = 0; jt < n && ok; ++jt) {
+      // Chunk of key tile jt and the tile's row offset inside that chunk.
+      int c = 0;
 #pragma unroll
-        for (int cc = 1; cc < kMaxChunks; ++cc) c += (jt >= kv.tile_start[cc]) ? 1 : 0;
-        const int row0 = (jt - kv.tile_start[c]) * kBN;
-        for (int t = 0; t < 2; ++t) {  // t = 0: K tile, t = 1: V tile
-          const int s = idx % kStages;
-          const uint32_t u = idx / kStages;
-          if (!mbar_wait(bar_kv_empty0 + 8 * s, (u & 1) ^ 1, abort_word, p.status, kStatusTimeout, lim)) {
-            ok = false;
-            break;
-          }
+      for (int cc = 1; cc < kMaxChunks; ++cc) c += (jt >= kv.tile_start[cc]) ? 1 : 0;
+      const int row0 = (jt - kv.tile_start[c]) * kBN;
+      for (int t = 0; t < 2; ++t) {  // t = 0: K tile, t = 1: V tile
+        const int s = idx % kStages;
+        const uint32_t u = idx / kStages;
+        const bool got = mbar_wait(bar_kv_empty0 + 8 * s, (u & 1) ^ 1, abort_word, p.status, kStatusTimeout, lim);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        if (leader) {
           const uint32_t full = bar_kv_full0 + 8 * s;
           mbar_arrive_expect_tx(full, L::kTileBytes);
           const CUtensorMap* map = t ? &kv.v[c] : &kv.k[c];
 #pragma unroll
           for (int b = 0; b < L::kBoxes; ++b)
             tma_load_3d(sRing + s * L::kTileBytes + b * L::kBoxBytes, map, full, b * 64, row0, bh);
-          ++idx;
         }
+        __syncwarp();
+        ++idx;
       }
-      if (!ok) {
-        // Aborted: let every copy already in flight land before the CTA exits.
-        // Slot s received ceil((idx - s) / kStages) loads; wait for the last.
-        for (int i = 0; i < kQTiles; ++i)
-          mbar_wait(bar_q_full0 + 8 * i, 0, nullptr, p.status, kStatusTimeout, lim);
-        for (int s = 0; s < kStages && s < idx; ++s) {
-          const int cnt = (idx - s + kStages - 1) / kStages;
-          mbar_wait(bar_kv_full0 + 8 * s, (cnt - 1) & 1, nullptr, p.status, kStatusTimeout, lim);
-        }
+    }
+    if (!ok) {
+      // Aborted: let every copy already in flight land before the CTA exits.
+      // Slot s received ceil((idx - s) / kStages) loads; wait for the last.
+      for (int i = 0; i < kQTiles; ++i)
+        mbar_wait(bar_q_full0 + 8 * i, 0, nullptr, p.status, kStatusTimeout, lim);
+      for (int s = 0; s < kStages && s < idx; ++s) {
+        const int cnt = (idx - s + kStages - 1) / kStages;
+        mbar_wait(bar_kv_full0 + 8 * s, (cnt - 1) & 1, nullptr, p.status, kStatusTimeout, lim);
       }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, kBN, false, false);
-      constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
-      const uint32_t tO0 = tmem + 2 * kBN;
+    // The whole warp runs the loop in step and waits on the barriers; the
+    // elected lane issues every tcgen05.mma and tcgen05.commit.  Shared-memory
+    // descriptors are built once and advanced by constant offsets.
+    const bool leader = elect_one();
+    constexpr uint32_t kIdS = idesc_bf16(128, kBN, false, false);
+    constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
+    constexpr uint64_t kTileDesc = L::kTileBytes >> 4;  // one tile in descriptor address units
+    const uint32_t tO0 = tmem + 2 * kBN;
+    const uint64_t dQ = sdesc_k_sw128(sQ);
+    const uint64_t dK = sdesc_k_sw128(sRing);
+    const uint64_t dV = sdesc_mn_sw128(sRing, L::kBoxBytes);
 
-      // S_i = Q_i K^T : K-major Q and K, 16 bf16 of depth per instruction.
-      auto issue_qk = [&](int i, uint32_t sK) {
-        const uint32_t sq = sQ + i * L::kTileBytes;
+    // S_i = Q_i K^T : K-major Q and K, 16 bf16 of depth per instruction
+    // (32 bytes inside a 128-byte row; the next 64 columns are the next box).
+    auto issue_qk = [&](int i, int slot) {
+      const uint64_t dq = dQ + i * kTileDesc, dk = dK + slot * kTileDesc;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * L::kBoxBytes + (kk % 4) * 32;
-          umma_ss(tmem + i * kBN, sdesc_k_sw128(sq + off), sdesc_k_sw128(sK + off), kIdS, kk > 0);
-        }
-      };
-      // O_i (+)= P_i V : P from TMEM (bf16 pairs, 8 columns per 16 keys),
-      // V MN-major (rows of 64 head-dim elements, 16 keys = 2048 bytes).
-      auto issue_pv = [&](int i, uint32_t sV, bool acc) {
+      for (int kk = 0; kk < D / 16; ++kk) {
+        constexpr int kBox = L::kBoxBytes;
+        const uint64_t off = static_cast<uint64_t>(((kk / 4) * kBox + (kk % 4) * 32) >> 4);
+        umma_ss(tmem + i * kBN, dq + off, dk + off, kIdS, kk > 0);
+      }
+    };
+    // O_i (+)= P_i V : P from TMEM (bf16 pairs, 8 columns per 16 keys),
+    // V MN-major (rows of 64 head-dim elements, 16 keys = 2048 bytes).
+    auto issue_pv = [&](int i, int slot, bool acc) {
+      const uint64_t dv = dV + slot * kTileDesc;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tO0 + i * D, tmem + i * kBN + kk * 8, sdesc_mn_sw128(sV + kk * 2048, L::kBoxBytes),
-                  kIdPV, (acc || kk > 0) ? 1u : 0u);
-      };
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        umma_ts(tO0 + i * D, tmem + i * kBN + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdPV,
+                (acc || kk > 0) ? 1u : 0u);
+    };
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      const bool got = PA_WAIT_HINT ? mbar_wait_hint(bar, parity, abort_word, p.status, kStatusTimeout, lim,
+                                                     kSuspendHintNs)
+                                    : mbar_wait(bar, parity, abort_word, p.status, kStatusTimeout, lim);
+      return __all_sync(0xffffffffu, got);
+    };
 
-      auto mma_wait = [&](uint32_t bar, uint32_t parity, volatile int* aw, int* st, int code, uint64_t limit) {
-        return PA_WAIT_HINT ? mbar_wait_hint(bar, parity, aw, st, code, limit, kSuspendHintNs)
-                            : mbar_wait(bar, parity, aw, st, code, limit);
-      };
-      bool ok = mbar_wait(bar_q_full0, 0, abort_word, p.status, kStatusTimeout, lim) &&
-                mbar_wait(bar_q_full0 + 8, 0, abort_word, p.status, kStatusTimeout, lim) &&
-                mbar_wait(bar_kv_full0, 0, abort_word, p.status, kStatusTimeout, lim);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, sRing);
+    bool ok = wait_all(bar_q_full0, 0) && wait_all(bar_q_full0 + 8, 0) && wait_all(bar_kv_full0, 0);
+    if (ok) {
+      tc_fence_after();
+      if (leader) {
+        issue_qk(0, 0);
         umma_commit(bar_s_full0);
-        issue_qk(1, sRing);
+        issue_qk(1, 0);
         umma_commit(bar_s_full0 + 8);
         umma_commit(bar_kv_empty0);
       }
-      int idx = 1;
-      for (int j = 0; j < n && ok; ++j) {
-        const int sv = idx % kStages;
-        const uint32_t uv = idx / kStages;
+      __syncwarp();
+    }
+    int idx = 1;
+    for (int j = 0; j < n && ok; ++j) {
+      const int sv = idx % kStages;
+      const uint32_t uv = idx / kStages;
+      ++idx;
+      int sk = 0;
+      uint32_t uk = 0;
+      const bool more = (j + 1 < n);
+      if (more) {
+        sk = idx % kStages;
+        uk = idx / kStages;
         ++idx;
-        int sk = 0;
-        uint32_t uk = 0;
-        const bool more = (j + 1 < n);
-        if (more) {
-          sk = idx % kStages;
-          uk = idx / kStages;
-          ++idx;
-        }
-        if (!mma_wait(bar_kv_full0 + 8 * sv, uv & 1, abort_word, p.status, kStatusTimeout, lim)) {
+      }
+      if (!wait_all(bar_kv_full0 + 8 * sv, uv & 1)) {
+        ok = false;
+        break;
+      }
+      for (int i = 0; i < 2; ++i) {
+        if (!wait_all(bar_p_full0 + 8 * i, j & 1)) {
           ok = false;
           break;
         }
-        for (int i = 0; i < 2; ++i) {
-          if (!mma_wait(bar_p_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(i, sRing + sv * L::kTileBytes, j > 0);
-          if (i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
-          if (more) {
-            if (i == 0) {
-              if (!mma_wait(bar_kv_full0 + 8 * sk, uk & 1, abort_word, p.status, kStatusTimeout, lim)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
+        tc_fence_after();
+        if (leader) issue_pv(i, sv, j > 0);
+        if (leader && i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
+        __syncwarp();
+        if (more) {
+          if (i == 0) {
+            if (!wait_all(bar_kv_full0 + 8 * sk, uk & 1)) {
+              ok = false;
+              break;
             }
-            issue_qk(i, sRing + sk * L::kTileBytes);
+            tc_fence_after();
+          }
+          if (leader) {
+            issue_qk(i, sk);
             umma_commit(bar_s_full0 + 8 * i);
             if (i == 1) umma_commit(bar_kv_empty0 + 8 * sk);
-          } else {
-            umma_commit(bar_o_full0 + 8 * i);
           }
+        } else if (leader) {
+          umma_commit(bar_o_full0 + 8 * i);
         }
+        __syncwarp();
       }
-      // Every MMA this thread issued completes before tensor memory is freed.
-      umma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
     }
+    // Every MMA issued completes before tensor memory is freed.
+    if (leader) umma_commit(bar_drain);
+    __syncwarp();
+    mbar_wait(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax

@@ -117,6 +117,20 @@ __device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, vo
   }
 }
 
+// One lane of the (fully converged) warp gets true.  A role whose loop the
+// whole warp runs in step issues its asynchronous instructions from this lane:
+// the loop's control flow stays warp-uniform, which keeps the issuing lane
+// from being starved of issue slots by busy warps on the same sub-partition.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Register re-allocation between warpgroups (whole warpgroup, immediate count).
 template <int kRegs>
 __device__ __forceinline__ void setmaxnreg_inc() {

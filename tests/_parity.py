@@ -38,8 +38,14 @@ def errors(o_gpu, lse_gpu, o_ref, lse_ref) -> dict:
     }
 
 
+# Every comparison made in this session, in order (written out by conftest.py
+# when PA_PARITY_REPORT names a file).
+RECORDED: list = []
+
+
 def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what: str = "") -> dict:
     e = errors(o_gpu, lse_gpu, o_ref, lse_ref)
+    RECORDED.append({"what": what, **e})
     msg = f"{what}: {e}"
     assert e["finite"], msg
     assert e["o_max_abs"] <= O_MAX_ABS, msg

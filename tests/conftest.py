@@ -1,3 +1,4 @@
+import json
 import os
 import sys
 
@@ -27,3 +28,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _parity_report():
+    """With PA_PARITY_REPORT=<path>, write every GPU-vs-oracle comparison of
+    the session (name, max-abs, mean-abs, relative L2, LSE relative error) to
+    that JSON file at the end."""
+    yield
+    path = os.environ.get("PA_PARITY_REPORT")
+    if path:
+        from tests import _parity
+        with open(path, "w") as f:
+            json.dump(_parity.RECORDED, f, indent=1)
