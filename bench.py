@@ -530,7 +530,7 @@ def extra_measurements(pa, device, peaks):
     """Secondary lines: the other workloads' device throughput (not the
     headline value).  Bounded repetitions each."""
     out = {}
-    plan = [("ring", 20, 3), ("tails", 10, 3), ("hunyuan", 3, 1)]
+    plan = [("ring", 20, 3), ("tails", 10, 3), ("flux1008", 10, 3), ("hunyuan", 3, 1)]
     for name, steps, warm in plan:
         w = workloads.get(name)
         r = time_workload(pa, w, steps, warm, device)
@@ -545,7 +545,7 @@ def extra_measurements(pa, device, peaks):
         ent["pct_of_bf16_peak"] = 100.0 * ent["fwd_tflops"] / peaks["bf16_tflops"]
         out[name] = ent
     # The chunked workloads as one fused launch (pa_attn_fwd_chunks).
-    for name in ("ring", "tails"):
+    for name in ("ring", "tails", "flux1008"):
         w = workloads.get(name)
         out[name + "_fused"] = fused_timing(pa, w, steps=20, warmup=3, device=device)
     out["hunyuan_8chunks_fused"] = fused_timing(

@@ -56,6 +56,14 @@ namespace single {
 #ifndef PA_SINGLE_EMU
 #define PA_SINGLE_EMU 0
 #endif
+//   PA_SPLIT_P        P handed to the MMA warp in this many parts (1, 2 or 4)
+//                     of the key tile, so P.V on the first parts runs while
+//                     the later ones are computed
+#ifndef PA_SPLIT_P
+#define PA_SPLIT_P 2
+#endif
+constexpr int kPParts = PA_SPLIT_P;
+static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P is handed over in 1, 2 or 4 parts");
 // Barrier waits:
 //   PA_WAIT_HINT      waits of the softmax warps and of the MMA-issuing thread
 //                     pass a long suspend-time hint to mbarrier.try_wait, so a
@@ -94,8 +102,9 @@ struct FwdLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kQTiles * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  // q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain,
+  // p_part[2][3] (parts of P before the last, which arrives on p_full)
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 6;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
   static constexpr int kBytes = kAbortOff + 4;
@@ -127,6 +136,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t bar_p_full0 = bars + 8 * (4 + 2 * kStages);
   const uint32_t bar_o_full0 = bars + 8 * (6 + 2 * kStages);
   const uint32_t bar_drain = bars + 8 * (8 + 2 * kStages);
+  const uint32_t bar_p_part0 = bars + 8 * (9 + 2 * kStages);  // + 8 * (3 * i + part)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kTmemSlotOff);
   volatile int* abort_word = reinterpret_cast<volatile int*>(gbase + L::kAbortOff);
 
@@ -146,6 +156,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_s_full0 + 8 * i, 1);
       mbar_init(bar_p_full0 + 8 * i, 4);  // one arrival per softmax warp
+      for (int q = 0; q < 3; ++q) mbar_init(bar_p_part0 + 8 * (3 * i + q), 4);
       mbar_init(bar_o_full0 + 8 * i, 1);
     }
     mbar_init(bar_drain, 1);
@@ -248,10 +259,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     };
     // O_i (+)= P_i V : P from TMEM (bf16 pairs, 8 columns per 16 keys),
     // V MN-major (rows of 64 head-dim elements, 16 keys = 2048 bytes).
-    auto issue_pv = [&](int i, int slot, bool acc) {
+    auto issue_pv = [&](int i, int slot, bool acc, int kk0 = 0, int kk1 = kBN / 16) {
       const uint64_t dv = dV + slot * kTileDesc;
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
+      for (int kk = kk0; kk < kk1; ++kk)
         umma_ts(tO0 + i * D, tmem + i * kBN + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdPV,
                 (acc || kk > 0) ? 1u : 0u);
     };
@@ -292,12 +303,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         break;
       }
       for (int i = 0; i < 2; ++i) {
-        if (!wait_all(bar_p_full0 + 8 * i, j & 1)) {
+        // P.V part by part: part q covers keys [q, q + 1) * kBN / kPParts.
+        constexpr int kKkPerPart = (kBN / 16) / kPParts;
+        for (int q = 0; q < kPParts - 1 && ok; ++q) {
+          if (!wait_all(bar_p_part0 + 8 * (3 * i + q), j & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (leader) issue_pv(i, sv, j > 0 || q > 0, q * kKkPerPart, (q + 1) * kKkPerPart);
+          __syncwarp();
+        }
+        if (!ok || !wait_all(bar_p_full0 + 8 * i, j & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (leader) issue_pv(i, sv, j > 0);
+        if (leader) issue_pv(i, sv, j > 0 || kPParts > 1, (kPParts - 1) * kKkPerPart, kBN / 16);
         if (leader && i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
         __syncwarp();
         if (more) {
@@ -434,6 +456,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st_x16(tS + ch * 16, pk);
+        constexpr int kChPerPart = (kBN / 32) / kPParts;  // 32-key chunks per part
+        if (kPParts > 1 && (ch + 1) % kChPerPart == 0 && ch + 1 < kBN / 32) {
+          // Part (ch + 1) / kChPerPart - 1 of P is in TMEM: hand it over.
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_p_part0 + 8 * (3 * i + (ch + 1) / kChPerPart - 1));
+        }
       }
 #if PA_SINGLE_F2
       {

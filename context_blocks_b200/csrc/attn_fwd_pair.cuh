@@ -168,7 +168,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // its own shared memory; the bytes are counted on the leader's barriers,
     // whose expected byte counts (set by the leader) cover both CTAs.
     // Ring order: K_0, V_0, K_1, V_1, ...; load idx goes to slot idx % kPairStages.
-    if (lane == 0) {
+    // The whole warp runs the loop in step; the elected lane issues.
+    const bool el = elect_one();
+    if (el) {
       for (int i = 0; i < kQTiles; ++i) {
         const uint32_t full = bar_q_full0 + 8 * i;
         if (leader) mbar_arrive_expect_tx(full, 2 * L::kQTileBytes);
@@ -177,16 +179,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int bx = 0; bx < 2; ++bx)
           tma_load_3d_pair(sQ + i * L::kQTileBytes + bx * L::kQBoxBytes, &tm_q, full_l, bx * 64, q0 + i * kBM, bh);
       }
-      bool ok = true;
-      int idx = 0;  // ring loads issued so far
-      for (int j = 0; j < n && ok; ++j) {
-        for (int t = 0; t < 2; ++t) {  // t = 0: K_j half, t = 1: V_j half
-          const int s = idx % kPairStages;
-          const uint32_t u = idx / kPairStages;
-          if (!mbar_wait_cluster(bar_kv_empty0 + 8 * s, (u & 1) ^ 1, abort_word, p.status, kStatusTimeout, lim)) {
-            ok = false;
-            break;
-          }
+    }
+    __syncwarp();
+    bool ok = true;
+    int idx = 0;  // ring loads issued so far
+    for (int j = 0; j < n && ok; ++j) {
+      for (int t = 0; t < 2; ++t) {  // t = 0: K_j half, t = 1: V_j half
+        const int s = idx % kPairStages;
+        const uint32_t u = idx / kPairStages;
+        const bool got =
+            mbar_wait_cluster(bar_kv_empty0 + 8 * s, (u & 1) ^ 1, abort_word, p.status, kStatusTimeout, lim);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        if (el) {
           const uint32_t full = bar_kv_full0 + 8 * s;
           if (leader) mbar_arrive_expect_tx(full, 2 * L::kSlotBytes);
           const uint32_t full_l = mapa_shared(full, 0);
@@ -201,122 +208,143 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // all 128 keys x head-dim columns [64 rank, +64) (one box)
             tma_load_3d_pair(dst, &tm_v, full_l, static_cast<int>(rank) * 64, j * kBN, bh);
           }
-          ++idx;
+        }
+        __syncwarp();
+        ++idx;
+      }
+    }
+    if (!ok) {
+      // Aborted.  The leader's barriers count both CTAs' bytes: the leader
+      // waits (bounded) for the last phase of each slot it armed; then both
+      // CTAs give straggling copies a further 200 us before leaving.
+      if (leader) {
+        for (int i = 0; i < kQTiles; ++i)
+          mbar_wait_cluster(bar_q_full0 + 8 * i, 0, nullptr, p.status, kStatusTimeout, lim);
+        for (int s = 0; s < kPairStages && s < idx; ++s) {
+          const int cnt = (idx - s + kPairStages - 1) / kPairStages;
+          mbar_wait_cluster(bar_kv_full0 + 8 * s, (cnt - 1) & 1, nullptr, p.status, kStatusTimeout, lim);
         }
       }
-      if (!ok) {
-        // Aborted.  The leader's barriers count both CTAs' bytes: the leader
-        // waits (bounded) for the last phase of each slot it armed; then both
-        // CTAs give straggling copies a further 200 us before leaving.
-        if (leader) {
-          for (int i = 0; i < kQTiles; ++i)
-            mbar_wait_cluster(bar_q_full0 + 8 * i, 0, nullptr, p.status, kStatusTimeout, lim);
-          for (int s = 0; s < kPairStages && s < idx; ++s) {
-            const int cnt = (idx - s + kPairStages - 1) / kPairStages;
-            mbar_wait_cluster(bar_kv_full0 + 8 * s, (cnt - 1) & 1, nullptr, p.status, kStatusTimeout, lim);
-          }
-        }
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 200000ull) {
-        }
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) {
       }
     }
     __syncwarp();
   } else if (leader && (warp == kMmaWarp || (kMmaThreads == 2 && warp == kMmaWarp + 2))) {
     // ------------------------------------------------------------ MMA issue
-    // Leader CTA only.  This thread serves query tiles [i_lo, i_hi): the pair
+    // Leader CTA only.  This warp serves query tiles [i_lo, i_hi): the pair
     // MMAs S_i = Q_i K_j^T and O_i += P_i V_j cover the Q_i rows of both CTAs
-    // (M = 256), each CTA's TMEM receiving its own 128 rows.
-    if (lane == 0) {
-      const int i_lo = (kMmaThreads == 2) ? (warp - kMmaWarp) / 2 : 0;
-      const int i_hi = (kMmaThreads == 2) ? i_lo + 1 : 2;
-      constexpr uint32_t kIdS = idesc_bf16(2 * kBM, kBN, false, false);
-      constexpr uint32_t kIdPV = idesc_bf16(2 * kBM, D, false, true);
+    // (M = 256), each CTA's TMEM receiving its own 128 rows.  The whole warp
+    // runs the loop in step; the elected lane issues.  Shared-memory
+    // descriptors are built once and advanced by constant offsets.
+    const bool el = elect_one();
+    const int i_lo = (kMmaThreads == 2) ? (warp - kMmaWarp) / 2 : 0;
+    const int i_hi = (kMmaThreads == 2) ? i_lo + 1 : 2;
+    constexpr uint32_t kIdS = idesc_bf16(2 * kBM, kBN, false, false);
+    constexpr uint32_t kIdPV = idesc_bf16(2 * kBM, D, false, true);
+    const uint64_t dQ = sdesc_k_sw128(sQ);
+    const uint64_t dK = sdesc_k_sw128(sRing);
+    const uint64_t dV = sdesc_mn_sw128(sRing, L::kSlotBytes);
 
-      // S_i = Q_i K^T : A = this CTA's Q_i (K-major, 16 KB per 64-column box),
-      // B = each CTA's 64 keys of K_j (K-major, 8 KB per 64-column box).
-      auto issue_qk = [&](int i, uint32_t sK) {
-        const uint32_t sQi = sQ + i * L::kQTileBytes;
+    // S_i = Q_i K^T : A = this CTA's Q_i (K-major, 16 KB per 64-column box),
+    // B = each CTA's 64 keys of K_j (K-major, 8 KB per 64-column box).
+    auto issue_qk = [&](int i, int slot) {
+      const uint64_t dq = dQ + static_cast<uint64_t>(i * (L::kQTileBytes >> 4));
+      const uint64_t dk = dK + static_cast<uint64_t>(slot * (L::kSlotBytes >> 4));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = sQi + (kk / 4) * L::kQBoxBytes + (kk % 4) * 32;
-          const uint32_t bb = sK + (kk / 4) * L::kKBoxBytes + (kk % 4) * 32;
-          umma_ss_pair(tmem + i * kBN, sdesc_k_sw128(a), sdesc_k_sw128(bb), kIdS, kk > 0);
-        }
-      };
-      // O_i (+)= P_i V, half h = keys [64h, 64h + 64): A = P_i in each CTA's
-      // TMEM (bf16 pairs, 8 columns per 16 keys); B = each CTA's 64 head-dim
-      // columns of V_j (MN-major, 16 keys = 2048 bytes).
-      auto issue_pv_half = [&](int i, uint32_t sV, int h, bool acc) {
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t oa = static_cast<uint64_t>(((kk / 4) * L::kQBoxBytes + (kk % 4) * 32) >> 4);
+        const uint64_t ob = static_cast<uint64_t>(((kk / 4) * L::kKBoxBytes + (kk % 4) * 32) >> 4);
+        umma_ss_pair(tmem + i * kBN, dq + oa, dk + ob, kIdS, kk > 0);
+      }
+    };
+    // O_i (+)= P_i V, half h = keys [64h, 64h + 64): A = P_i in each CTA's
+    // TMEM (bf16 pairs, 8 columns per 16 keys); B = each CTA's 64 head-dim
+    // columns of V_j (MN-major, 16 keys = 2048 bytes).
+    auto issue_pv_half = [&](int i, int slot, int h, bool acc) {
+      const uint64_t dv = dV + static_cast<uint64_t>(slot * (L::kSlotBytes >> 4));
 #pragma unroll
-        for (int q = 0; q < kBN / 32; ++q) {
-          const int kk = h * (kBN / 32) + q;
-          umma_ts_pair(tmem + 2 * kBN + i * D, tmem + i * kBN + kk * 8, sdesc_mn_sw128(sV + kk * 2048, L::kSlotBytes),
-                       kIdPV, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
+      for (int q = 0; q < kBN / 32; ++q) {
+        const int kk = h * (kBN / 32) + q;
+        umma_ts_pair(tmem + 2 * kBN + i * D, tmem + i * kBN + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)),
+                     kIdPV, (acc || kk > 0) ? 1u : 0u);
+      }
+    };
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      const bool got = mbar_wait_cluster(bar, parity, abort_word, p.status, kStatusTimeout, lim);
+      return __all_sync(0xffffffffu, got);
+    };
 
-      bool ok = mbar_wait_cluster(bar_kv_full0, 0, abort_word, p.status, kStatusTimeout, lim);
-      for (int i = i_lo; i < i_hi && ok; ++i) {
-        ok = mbar_wait_cluster(bar_q_full0 + 8 * i, 0, abort_word, p.status, kStatusTimeout, lim);
-        if (ok) {
-          tc_fence_after();
-          issue_qk(i, sRing);
+    bool ok = wait_all(bar_kv_full0, 0);
+    for (int i = i_lo; i < i_hi && ok; ++i) {
+      ok = wait_all(bar_q_full0 + 8 * i, 0);
+      if (ok) {
+        tc_fence_after();
+        if (el) {
+          issue_qk(i, 0);
           umma_commit_pair_both(bar_s_full0 + 8 * i);
         }
+        __syncwarp();
       }
-      if (ok) umma_commit_pair_both(bar_kv_empty0);
-      int idx = 1;  // ring position of the next tile to consume (K0 was 0)
-      for (int j = 0; j < n && ok; ++j) {
-        const int sv = idx % kPairStages;
-        const uint32_t uv = idx / kPairStages;
+    }
+    if (ok && el) umma_commit_pair_both(bar_kv_empty0);
+    __syncwarp();
+    int idx = 1;  // ring position of the next tile to consume (K0 was 0)
+    for (int j = 0; j < n && ok; ++j) {
+      const int sv = idx % kPairStages;
+      const uint32_t uv = idx / kPairStages;
+      ++idx;
+      int sk = 0;
+      uint32_t uk = 0;
+      const bool more = (j + 1 < n);
+      if (more) {
+        sk = idx % kPairStages;
+        uk = idx / kPairStages;
         ++idx;
-        int sk = 0;
-        uint32_t uk = 0;
-        const bool more = (j + 1 < n);
-        if (more) {
-          sk = idx % kPairStages;
-          uk = idx / kPairStages;
-          ++idx;
-        }
-        if (!mbar_wait_cluster(bar_kv_full0 + 8 * sv, uv & 1, abort_word, p.status, kStatusTimeout, lim)) {
-          ok = false;
-          break;
-        }
-        for (int i = i_lo; i < i_hi && ok; ++i) {
-          // O_i += P_i V_j in two halves: the first half of P is ready while
-          // the softmax warpgroups still compute the second.
-          for (int h = 0; h < 2 && ok; ++h) {
-            ok = mbar_wait_cluster(bar_p_full0 + 8 * (2 * i + h), j & 1, abort_word, p.status, kStatusTimeout, lim);
-            if (ok) {
-              tc_fence_after();
-              issue_pv_half(i, sRing + sv * L::kSlotBytes, h, j > 0);
-            }
+      }
+      if (!wait_all(bar_kv_full0 + 8 * sv, uv & 1)) {
+        ok = false;
+        break;
+      }
+      for (int i = i_lo; i < i_hi && ok; ++i) {
+        // O_i += P_i V_j in two halves: the first half of P is ready while
+        // the softmax warpgroups still compute the second.
+        for (int h = 0; h < 2 && ok; ++h) {
+          ok = wait_all(bar_p_full0 + 8 * (2 * i + h), j & 1);
+          if (ok) {
+            tc_fence_after();
+            if (el) issue_pv_half(i, sv, h, j > 0);
+            __syncwarp();
           }
-          if (!ok) break;
-          if (i == i_hi - 1) umma_commit_pair_both(bar_kv_empty0 + 8 * sv);
-          if (more) {
-            if (i == i_lo) {
-              if (!mbar_wait_cluster(bar_kv_full0 + 8 * sk, uk & 1, abort_word, p.status, kStatusTimeout, lim)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
+        }
+        if (!ok) break;
+        if (el && i == i_hi - 1) umma_commit_pair_both(bar_kv_empty0 + 8 * sv);
+        __syncwarp();
+        if (more) {
+          if (i == i_lo) {
+            if (!wait_all(bar_kv_full0 + 8 * sk, uk & 1)) {
+              ok = false;
+              break;
             }
-            // S_i(j+1) overwrites the columns P_i(j) occupies: issued after
-            // the P.V that reads them, and MMAs of one thread run in order.
-            issue_qk(i, sRing + sk * L::kSlotBytes);
+            tc_fence_after();
+          }
+          // S_i(j+1) overwrites the columns P_i(j) occupies: issued after
+          // the P.V that reads them, and MMAs of one thread run in order.
+          if (el) {
+            issue_qk(i, sk);
             umma_commit_pair_both(bar_s_full0 + 8 * i);
             if (i == i_hi - 1) umma_commit_pair_both(bar_kv_empty0 + 8 * sk);
-          } else {
-            umma_commit_pair_both(bar_o_full0 + 8 * i);
           }
+        } else if (el) {
+          umma_commit_pair_both(bar_o_full0 + 8 * i);
         }
+        __syncwarp();
       }
-      // Every MMA this thread issued completes before tensor memory is freed.
-      umma_commit_pair_both(bar_drain);
-      mbar_wait_cluster(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
     }
+    // Every MMA this warp issued completes before tensor memory is freed.
+    if (el) umma_commit_pair_both(bar_drain);
+    __syncwarp();
+    mbar_wait_cluster(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax

@@ -370,6 +370,13 @@ def test_fused_hunyuan_eight_chunks(pa):
     _fused_check(pa, w, rows=_hunyuan_rows(w))
 
 
+def test_flux_1008_ring_anything(pa):
+    # per-chunk forward + merge, and the same chunks in one fused launch
+    w = workloads.get("flux1008")
+    _check_workload(pa, w)
+    _fused_check(pa, w)
+
+
 def test_fused_rejects_more_than_eight_chunks(pa):
     q = torch.zeros((1, 1, 8, 128), dtype=torch.bfloat16, device="cuda")
     ks = [torch.zeros((1, 1, 4, 128), dtype=torch.bfloat16, device="cuda") for _ in range(9)]

@@ -4,7 +4,7 @@ This module holds shapes, seeds and random draws only: none of the attention
 arithmetic lives here, so both the CUDA path and the oracle can take their
 inputs from it without sharing any of the method.
 
-The five workloads stand in for the attention calls of the two models the
+The workloads stand in for the attention calls of the two models the
 diffusers "ParaAttention" guide times (FLUX.1-dev at 1024x1024: 512 text +
 4096 image tokens, 24 heads of 128; HunyuanVideo at 720p, 129 frames:
 33 x 45 x 80 latent tokens + 256 text tokens) and for the ring-attention
@@ -67,6 +67,14 @@ WORKLOADS: Dict[str, Workload] = {
     "hunyuan": Workload("hunyuan", B=1, H=24, Nq=119056, Nk=119056, d=128, rms_qk=True,
                         chunks=(119056,), seed=4,
                         note="HunyuanVideo 720p x 129 frames: 33*45*80 video + 256 text tokens"),
+    # FLUX.1-dev at 1008 x 1008: 63 * 63 = 3969 image tokens + 512 text tokens
+    # = 4481, a length that does not divide by 4 ranks.  Split the way
+    # "Ring Anything Attention" of the "Context parallelism" guide does it:
+    # each rank holds ceil(4481 / 4) = 1121 tokens, the last one 1118 once the
+    # padding is trimmed before attention.
+    "flux1008": Workload("flux1008", B=1, H=24, Nq=4481, Nk=4481, d=128, rms_qk=True,
+                         chunks=(1121, 1121, 1121, 1118), seed=5,
+                         note="FLUX.1-dev 1008^2: 512 text + 3969 image tokens, ring-anything split over 4"),
 }
 
 # The 8-chunk split of the HunyuanVideo-shaped workload (ring_degree = 8).
