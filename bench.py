@@ -46,8 +46,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
 # kernel source whose digest is recorded with it.  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "78be64cc02328ba1230744048d229611863726660ed9f164ca1ce5daaeef77c0",
-    "bytes_per_launch": 84989952 + 5036288,   # dram__bytes_read.sum + dram__bytes_write.sum
+    "source_sha256": "2d699bce6e69f80019558ded24ecc2ac48f03bbf9c792d67057c5fa1b7608e43",
+    "bytes_per_launch": 84987904 + 11835648,   # dram__bytes_read.sum + dram__bytes_write.sum
     "capture": "profiles/attn_fwd_flux.md",
 }
 
