@@ -526,6 +526,32 @@ def fused_timing(pa, w, steps, warmup, device):
     return {"step_ms": ms, "tflops_step": fl / (ms * 1e-3) / 1e12, "launches_per_step": 1}
 
 
+def fp8_timing(pa, w, steps, warmup, device):
+    """Device time of pa_attn_fwd_fp8 on the workload's inputs quantised to
+    per-tensor scaled e4m3 (the quantisation is outside the timed region)."""
+    import torch
+    q, k, v = workloads.make_case(w, device=device)
+    qs = []
+    for x in (q, k, v):
+        sc = max(float(x.float().abs().max()), 1e-12) / 448.0
+        qs.append(((x.float() / sc).to(torch.float8_e4m3fn).contiguous(), sc))
+    del q, k, v
+    (q8, sq), (k8, sk), (v8, sv) = qs
+    o = torch.empty(q8.shape, dtype=torch.bfloat16, device=device)
+    lse = torch.empty(q8.shape[:3], dtype=torch.float32, device=device)
+    for _ in range(warmup):
+        pa.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, scale=w.scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        pa.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, scale=w.scale, out=o, lse=lse)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    return ms, workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d) / (ms * 1e-3) / 1e12
+
+
 def extra_measurements(pa, device, peaks):
     """Secondary lines: the other workloads' device throughput (not the
     headline value).  Bounded repetitions each."""
@@ -550,6 +576,13 @@ def extra_measurements(pa, device, peaks):
         out[name + "_fused"] = fused_timing(pa, w, steps=20, warmup=3, device=device)
     out["hunyuan_8chunks_fused"] = fused_timing(
         pa, workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8), steps=2, warmup=1, device=device)
+    # The e4m3 forward on the FLUX and HunyuanVideo shapes; its peak is the
+    # measured bf16 burst figure times the nominal fp8/bf16 ratio of 2.
+    for name, steps in (("flux", 20), ("hunyuan", 2)):
+        ms, tf = fp8_timing(pa, workloads.get(name), steps=steps, warmup=2, device=device)
+        out[name + "_fp8"] = {"fwd_ms_per_launch": ms, "fwd_tflops": tf,
+                              "frac_of_fp8_peak": tf / (2.0 * peaks["bf16_tflops"]),
+                              "peak_basis": "2 x measured bf16 burst (nominal e4m3/bf16 ratio)"}
     # The CTA-pair forward kernel (pa_attn_fwd_pair) on the FLUX-shaped workload.
     wf = workloads.get("flux")
     r = time_workload(pa, wf, 200, 10, device, pair=True)

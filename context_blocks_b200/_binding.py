@@ -30,6 +30,7 @@ _VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "pa_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_fwd_pair": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
+    "pa_attn_fwd_fp8": (_I, [_VP, _VP, _VP, _F, _F, _F, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_fwd_chunks": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _VP]),
     "pa_attn_chunks_noalloc": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
@@ -143,6 +144,35 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=
     rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
             float(scale), _stream_handle(stream, q.device))
     _check(rc, "pa_attn_fwd_pair" if pair else "pa_attn_fwd")
+    return out, lse
+
+
+def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, scale: Optional[float] = None,
+                 out=None, lse=None, stream=None):
+    """Attention over e4m3 inputs (``pa_attn_fwd_fp8``): q [B,H,Nq,128],
+    k, v [B,H,Nk,128] of dtype torch.float8_e4m3fn, whose real values are the
+    tensors times their scales.  Returns (o bf16, lse fp32) like attn_fwd."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float8_e4m3fn:
+            raise TypeError(f"{name} must be a torch.float8_e4m3fn tensor")
+        if t.device.type != "cuda" or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-d CUDA tensor")
+    B, H, Nq, d = q.shape
+    if k.shape[:2] != (B, H) or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    else:
+        _check_bf16("out", out, 4)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    rc = load_library().pa_attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
+                                        float(v_scale), out.data_ptr(), lse.data_ptr(), B, H, Nq, k.shape[2], d,
+                                        float(scale), _stream_handle(stream, q.device))
+    _check(rc, "pa_attn_fwd_fp8")
     return out, lse
 
 

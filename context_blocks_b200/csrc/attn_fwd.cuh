@@ -93,11 +93,17 @@ constexpr int kFwdThreads = 320;   // 10 warps
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
 
-template <int D>
+// kFp8: Q, K, V are e4m3 (one byte per element) instead of bf16.
+template <int D, bool kFp8 = false>
 struct FwdLayout {
   static_assert(D == 64 || D == 128, "head dim must be 64 or 128");
-  static constexpr int kBoxBytes = 128 * 128;        // 128 rows x 64 bf16, 128B-swizzled
-  static constexpr int kBoxes = D / 64;
+  static_assert(!kFp8 || D == 128, "the e4m3 path is written for d = 128 (one 128-byte row per key)");
+  static constexpr int kElemBytes = kFp8 ? 1 : 2;
+  static constexpr int kBoxCols = 128 / kElemBytes;  // elements in one 128-byte swizzled row
+  static constexpr int kBoxBytes = 128 * 128;        // 128 rows x 128 bytes, 128B-swizzled
+  static constexpr int kBoxes = D / kBoxCols;
+  // Contraction depth of one MMA: 32 bytes = 16 bf16 or 32 e4m3 elements.
+  static constexpr int kKPerMma = kFp8 ? 32 : 16;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row tile of Q, K or V
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kQTiles * kTileBytes;
@@ -116,11 +122,13 @@ struct FwdLayout {
       (kBytes + 1024 > kMinOneCtaPerSm) ? (kBytes + 1024) : kMinOneCtaPerSm;
 };
 
-template <int D>
+template <int D, bool kFp8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ KvChunks kv,
                     const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, kFp8>;
+  // Contraction depth of one MMA: 16 bf16 or 32 e4m3 elements (32 bytes).
+  constexpr int kKPerMma = kFp8 ? 32 : 16;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_arrive_expect_tx(bar_q_full0 + 8 * i, L::kTileBytes);
 #pragma unroll
         for (int b = 0; b < L::kBoxes; ++b)
-          tma_load_3d(sQ + i * L::kTileBytes + b * L::kBoxBytes, &tm_q, bar_q_full0 + 8 * i, b * 64,
+          tma_load_3d(sQ + i * L::kTileBytes + b * L::kBoxBytes, &tm_q, bar_q_full0 + 8 * i, b * L::kBoxCols,
                       q0 + i * kBM, bh);
       }
     }
@@ -215,7 +223,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const CUtensorMap* map = t ? &kv.v[c] : &kv.k[c];
 #pragma unroll
           for (int b = 0; b < L::kBoxes; ++b)
-            tma_load_3d(sRing + s * L::kTileBytes + b * L::kBoxBytes, map, full, b * 64, row0, bh);
+            tma_load_3d(sRing + s * L::kTileBytes + b * L::kBoxBytes, map, full, b * L::kBoxCols, row0, bh);
         }
         __syncwarp();
         ++idx;
@@ -238,33 +246,43 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // elected lane issues every tcgen05.mma and tcgen05.commit.  Shared-memory
     // descriptors are built once and advanced by constant offsets.
     const bool leader = elect_one();
-    constexpr uint32_t kIdS = idesc_bf16(128, kBN, false, false);
-    constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
+    constexpr uint32_t kIdS = kFp8 ? idesc_e4m3(128, kBN, false) : idesc_bf16(128, kBN, false, false);
+    constexpr uint32_t kIdPV = kFp8 ? idesc_e4m3(128, D, true) : idesc_bf16(128, D, false, true);
     constexpr uint64_t kTileDesc = L::kTileBytes >> 4;  // one tile in descriptor address units
     const uint32_t tO0 = tmem + 2 * kBN;
     const uint64_t dQ = sdesc_k_sw128(sQ);
     const uint64_t dK = sdesc_k_sw128(sRing);
     const uint64_t dV = sdesc_mn_sw128(sRing, L::kBoxBytes);
 
-    // S_i = Q_i K^T : K-major Q and K, 16 bf16 of depth per instruction
-    // (32 bytes inside a 128-byte row; the next 64 columns are the next box).
+    // S_i = Q_i K^T : K-major Q and K, 32 bytes of depth per instruction (16
+    // bf16 or 32 e4m3) inside a 128-byte row; the next row's worth of head
+    // dimension is the next box.
     auto issue_qk = [&](int i, int slot) {
       const uint64_t dq = dQ + i * kTileDesc, dk = dK + slot * kTileDesc;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
+      for (int kk = 0; kk < D / kKPerMma; ++kk) {
         constexpr int kBox = L::kBoxBytes;
         const uint64_t off = static_cast<uint64_t>(((kk / 4) * kBox + (kk % 4) * 32) >> 4);
-        umma_ss(tmem + i * kBN, dq + off, dk + off, kIdS, kk > 0);
+        if constexpr (kFp8)
+          umma_ss_f8(tmem + i * kBN, dq + off, dk + off, kIdS, kk > 0);
+        else
+          umma_ss(tmem + i * kBN, dq + off, dk + off, kIdS, kk > 0);
       }
     };
     // O_i (+)= P_i V : P from TMEM (bf16 pairs, 8 columns per 16 keys),
     // V MN-major (rows of 64 head-dim elements, 16 keys = 2048 bytes).
-    auto issue_pv = [&](int i, int slot, bool acc, int kk0 = 0, int kk1 = kBN / 16) {
+    // P occupies 8 TMEM columns per MMA (16 bf16 or 32 e4m3 keys); V is
+    // MN-major, one MMA's keys = kKPerMma rows of 128 bytes.
+    auto issue_pv = [&](int i, int slot, bool acc, int kk0 = 0, int kk1 = kBN / L::kKPerMma) {
       const uint64_t dv = dV + slot * kTileDesc;
 #pragma unroll
-      for (int kk = kk0; kk < kk1; ++kk)
-        umma_ts(tO0 + i * D, tmem + i * kBN + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdPV,
-                (acc || kk > 0) ? 1u : 0u);
+      for (int kk = kk0; kk < kk1; ++kk) {
+        const uint64_t voff = static_cast<uint64_t>(kk * ((kKPerMma * 128) >> 4));
+        if constexpr (kFp8)
+          umma_ts_f8(tO0 + i * D, tmem + i * kBN + kk * 8, dv + voff, kIdPV, (acc || kk > 0) ? 1u : 0u);
+        else
+          umma_ts(tO0 + i * D, tmem + i * kBN + kk * 8, dv + voff, kIdPV, (acc || kk > 0) ? 1u : 0u);
+      }
     };
     auto wait_all = [&](uint32_t bar, uint32_t parity) {
       const bool got = PA_WAIT_HINT ? mbar_wait_hint(bar, parity, abort_word, p.status, kStatusTimeout, lim,
@@ -304,7 +322,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       for (int i = 0; i < 2; ++i) {
         // P.V part by part: part q covers keys [q, q + 1) * kBN / kPParts.
-        constexpr int kKkPerPart = (kBN / 16) / kPParts;
+        constexpr int kKkPerPart = (kBN / kKPerMma) / kPParts;
         for (int q = 0; q < kPParts - 1 && ok; ++q) {
           if (!wait_all(bar_p_part0 + 8 * (3 * i + q), j & 1)) {
             ok = false;
@@ -319,7 +337,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           break;
         }
         tc_fence_after();
-        if (leader) issue_pv(i, sv, j > 0 || kPParts > 1, (kPParts - 1) * kKkPerPart, kBN / 16);
+        if (leader) issue_pv(i, sv, j > 0 || kPParts > 1, (kPParts - 1) * kKkPerPart, kBN / kKPerMma);
         if (leader && i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
         __syncwarp();
         if (more) {
@@ -453,9 +471,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           l += p0 + p1;
 #endif
-          pk[e] = pack_bf16x2(p0, p1);
+          if constexpr (kFp8) {
+            // four e4m3 keys per 32-bit column, lowest key in the low byte
+            const uint32_t h = pack_e4m3x2(p0, p1);
+            if (e & 1)
+              pk[e >> 1] |= h << 16;
+            else
+              pk[e >> 1] = h;
+          } else {
+            pk[e] = pack_bf16x2(p0, p1);
+          }
         }
-        tmem_st_x16(tS + ch * 16, pk);
+        if constexpr (kFp8) {
+          const uint32_t(&pk8)[8] = *reinterpret_cast<const uint32_t(*)[8]>(pk);
+          tmem_st_x8(tS + ch * 8, pk8);
+        } else {
+          tmem_st_x16(tS + ch * 16, pk);
+        }
         constexpr int kChPerPart = (kBN / 32) / kPParts;  // 32-key chunks per part
         if (kPParts > 1 && (ch + 1) % kChPerPart == 0 && ch + 1 < kBN / 32) {
           // Part (ch + 1) / kChPerPart - 1 of P is in TMEM: hand it over.
@@ -485,7 +517,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = p.o_scale / l;
       const bool in_range = row < p.Nq;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.Nq + row) * D;
 #pragma unroll

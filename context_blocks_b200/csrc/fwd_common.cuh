@@ -30,6 +30,7 @@ struct FwdParams {
   float scale_log2;     // scale * log2(e)
   int* status;          // device status word
   unsigned long long timeout_ns;
+  float o_scale;        // O is multiplied by this (the V dequantisation scale; 1 for bf16)
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -68,7 +68,7 @@ struct DeviceState {
   int sm_count = 0;
   int* status = nullptr;  // device address of pa::g_status
   unsigned char* noalloc_scratch = nullptr;  // device address of pa::g_noalloc_scratch
-  bool fwd_attr[2] = {false, false};
+  bool fwd_attr[3] = {false, false, false};  // d = 64, d = 128, e4m3 d = 128
   bool pair_attr = false;
 };
 
@@ -147,16 +147,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 3-D map over a [BH, N, d] bf16 tensor: box of 64 head-dim elements x
 // box_rows rows x 1, 128-byte swizzle, zero fill outside the tensor.
-int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int box_rows) {
+// 3-D map (d, N, B*H) with 128-byte swizzled boxes of one 128-byte row of d by
+// box_rows rows: 64 bf16 or (fp8) 128 one-byte elements per row.
+int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int box_rows, bool fp8 = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  const int eb = fp8 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n_rows),
                         static_cast<cuuint64_t>(bh)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                           static_cast<cuuint64_t>(n_rows) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb,
+                           static_cast<cuuint64_t>(n_rows) * static_cast<cuuint64_t>(d) * eb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+  CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(ptr), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
@@ -164,18 +168,21 @@ int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int
 }
 
 // Single-CTA forward over n_chunks K/V chunks (n_chunks = 1 for one chunk).
-template <int D>
+// kFp8: e4m3 Q/K/V with dequantisation scales; qk_scale multiplies the logits
+// (on top of `scale`) and o_scale the output.
+template <int D, bool kFp8 = false>
 int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void* const* v, const int* nk,
-               int n_chunks, void* o, float* lse, int BH, int Nq, float scale, cudaStream_t stream) {
-  using L = pa::single::FwdLayout<D>;
+               int n_chunks, void* o, float* lse, int BH, int Nq, float scale, cudaStream_t stream,
+               float qk_scale = 1.f, float o_scale = 1.f) {
+  using L = pa::single::FwdLayout<D, kFp8>;
   CUtensorMap tq;
   pa::single::KvChunks kv;
   int rc;
-  if ((rc = encode_map(&tq, q, D, Nq, BH, pa::kBM)) != PA_OK) return rc;
+  if ((rc = encode_map(&tq, q, D, Nq, BH, pa::kBM, kFp8)) != PA_OK) return rc;
   long long nk_total = 0, tiles_total = 0;
   for (int c = 0; c < n_chunks; ++c) {
-    if ((rc = encode_map(&kv.k[c], k[c], D, nk[c], BH, pa::kBN)) != PA_OK) return rc;
-    if ((rc = encode_map(&kv.v[c], v[c], D, nk[c], BH, pa::kBN)) != PA_OK) return rc;
+    if ((rc = encode_map(&kv.k[c], k[c], D, nk[c], BH, pa::kBN, kFp8)) != PA_OK) return rc;
+    if ((rc = encode_map(&kv.v[c], v[c], D, nk[c], BH, pa::kBN, kFp8)) != PA_OK) return rc;
     kv.nk[c] = nk[c];
     kv.tiles[c] = (nk[c] + pa::kBN - 1) / pa::kBN;
     kv.tile_start[c] = static_cast<int>(tiles_total);
@@ -189,8 +196,8 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   }
   kv.n_chunks = n_chunks;
   if (nk_total > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "more than 2^31 keys in one call");
-  auto kern = pa::single::attn_fwd_kernel<D>;
-  const int slot = (D == 64) ? 0 : 1;
+  auto kern = pa::single::attn_fwd_kernel<D, kFp8>;
+  const int slot = kFp8 ? 2 : (D == 64) ? 0 : 1;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!st->fwd_attr[slot]) {
@@ -205,9 +212,10 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   prm.Nq = Nq;
   prm.Nk = static_cast<int>(nk_total);
   prm.n_kv_tiles = static_cast<int>(tiles_total);
-  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.scale_log2 = scale * qk_scale * 1.4426950408889634f;
   prm.status = st->status;
   prm.timeout_ns = kDefaultTimeoutNs;
+  prm.o_scale = o_scale;
   dim3 grid((Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM), BH);
   kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, kv, prm);
   cudaError_t e = cudaGetLastError();
@@ -250,6 +258,7 @@ int launch_fwd_pair(DeviceState* st, const void* q, const void* k, const void* v
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.status = st->status;
   prm.timeout_ns = kDefaultTimeoutNs;
+  prm.o_scale = 1.f;
   const int rows_per_pair = 2 * pa::kQTiles * pa::kBM;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ((Nq + rows_per_pair - 1) / rows_per_pair), BH);
@@ -292,7 +301,7 @@ namespace {
 // Argument checks shared by the forward entry points.  On PA_OK, *st is the
 // current device's state, or null when there is nothing to do (Nq == 0).
 int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
-                   int d, float scale, DeviceState** st, bool host_only = false) {
+                   int d, float scale, DeviceState** st, bool host_only = false, int in_elem_bytes = 2) {
   *st = nullptr;
   if (!q || !k || !v || !o || !lse) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
   if (B < 1 || H < 1) return fail(PA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
@@ -306,15 +315,16 @@ int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* 
     return fail(PA_ERR_MISALIGNED, "q, k, v and o must be 16-byte aligned");
   if (!aligned(lse, 4)) return fail(PA_ERR_MISALIGNED, "lse must be 4-byte aligned");
   if (Nq == 0) return PA_OK;
-  const uint64_t qbytes = static_cast<uint64_t>(bh) * Nq * d * 2;
-  const uint64_t kbytes = static_cast<uint64_t>(bh) * Nk * d * 2;
+  const uint64_t qbytes = static_cast<uint64_t>(bh) * Nq * d * in_elem_bytes;
+  const uint64_t kbytes = static_cast<uint64_t>(bh) * Nk * d * in_elem_bytes;
+  const uint64_t obytes = static_cast<uint64_t>(bh) * Nq * d * 2;
   const uint64_t lbytes = static_cast<uint64_t>(bh) * Nq * 4;
   const void* ins[3] = {q, k, v};
   const uint64_t in_bytes[3] = {qbytes, kbytes, kbytes};
   for (int i = 0; i < 3; ++i)
-    if (overlap(ins[i], in_bytes[i], o, qbytes) || overlap(ins[i], in_bytes[i], lse, lbytes))
+    if (overlap(ins[i], in_bytes[i], o, obytes) || overlap(ins[i], in_bytes[i], lse, lbytes))
       return fail(PA_ERR_INVALID_ARG, "outputs overlap an input");
-  if (overlap(o, qbytes, lse, lbytes)) return fail(PA_ERR_INVALID_ARG, "o and lse overlap");
+  if (overlap(o, obytes, lse, lbytes)) return fail(PA_ERR_INVALID_ARG, "o and lse overlap");
   if (host_only) return PA_OK;
 
   (void)cudaGetLastError();
@@ -339,6 +349,21 @@ int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64) return launch_fwd<64>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, s);
   return launch_fwd<128>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, s);
+}
+
+int pa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale, float v_scale,
+                    void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale, void* stream) {
+  g_err[0] = '\0';
+  for (float sc : {q_scale, k_scale, v_scale})
+    if (!std::isfinite(sc) || !(sc > 0.f)) return fail(PA_ERR_INVALID_ARG, "dequantisation scales must be finite and > 0");
+  DeviceState* st = nullptr;
+  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, true, 1);  // host-side checks
+  if (rc != PA_OK) return rc;
+  if (d != 128) return fail(PA_ERR_UNSUPPORTED, "the e4m3 forward needs d = 128 (got %d)", d);
+  rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, false, 1);
+  if (rc != PA_OK || st == nullptr) return rc;
+  return launch_fwd<128, true>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, static_cast<cudaStream_t>(stream),
+                               q_scale * k_scale, v_scale);
 }
 
 int pa_attn_fwd_chunks(const void* q, const void* const* k_chunks, const void* const* v_chunks,

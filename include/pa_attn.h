@@ -82,6 +82,32 @@ int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
                 int Nq, int Nk, int d, float scale, void* stream);
 
 /*
+ * pa_attn_fwd_fp8 - pa_attn_fwd with e4m3 (fp8) Q, K and V.
+ *
+ * The pages' fp8 path quantises activations dynamically to fp8 (diffusers
+ * "ParaAttention" guide, fp8 section); this entry applies the same storage
+ * format to the attention inputs.  Each input is one scaled e4m3 tensor:
+ *     q_real = q_scale * decode(q),  k_real = k_scale * decode(k),
+ *     v_real = v_scale * decode(v)              (decode: OCP E4M3FN)
+ * and o, lse are the attention of pa_attn_fwd over q_real, k_real, v_real.
+ * Q.K^T and P.V run on the tensor cores in e4m3 with fp32 accumulation; the
+ * softmax is fp32 and P is rounded to e4m3 (range 2^-9 .. 448) before P.V,
+ * which is the dominant error: about 2^-4 relative per weight.
+ *
+ * q        [B,H,Nq,d] e4m3 (1 byte), device, 16-byte aligned     (input)
+ * k, v     [B,H,Nk,d] e4m3, device, 16-byte aligned              (input)
+ * q_scale, k_scale, v_scale   finite and > 0
+ * o        [B,H,Nq,d] bf16; lse [B,H,Nq] fp32                      (outputs)
+ * d        128 only (PA_ERR_UNSUPPORTED otherwise)
+ * B, H, Nq, Nk, scale, stream   as pa_attn_fwd
+ *
+ * Errors: as pa_attn_fwd; PA_ERR_INVALID_ARG for a bad scale.
+ */
+int pa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale,
+                    float v_scale, void* o, float* lse, int B, int H, int Nq, int Nk, int d,
+                    float scale, void* stream);
+
+/*
  * pa_attn_fwd_chunks - attention of Q over several K/V chunks in one launch.
  *
  * The local loop of Ring Attention fused (diffusers "Context parallelism",

@@ -38,6 +38,18 @@ def errors(o_gpu, lse_gpu, o_ref, lse_ref) -> dict:
     }
 
 
+# e4m3 forward (pa_attn_fwd_fp8), against the oracle on the dequantised inputs.
+# The inputs' own quantisation is exact on both sides; what remains is P
+# rounded to e4m3 before P.V: a relative error of at most 2^-4 per weight,
+# about 2^-4/sqrt(3) = 3.6% rms.  So O's error is bounded elementwise by
+# 2^-4 * sum_j w_j |v_j| <= 2^-4 max|v| (plus the bf16 rounding of O,
+# 2^-8 max|o| with margin), and on average it is a few per cent of |o|.  The
+# bounds are therefore relative: relative L2 <= 6e-2, mean-abs <= 6e-2 of the
+# mean |o_ref|, max-abs <= 2^-4 max|v| + 2^-8 max|o_ref|.  LSE uses the fp32
+# exponentials and keeps the bf16 bound.
+FP8_O_REL_L2 = 6e-2
+FP8_O_MEAN_REL = 6e-2
+
 # Every comparison made in this session, in order (written out by conftest.py
 # when PA_PARITY_REPORT names a file).
 RECORDED: list = []
@@ -52,4 +64,18 @@ def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what: str = "") -> dict:
     assert e["o_mean_abs"] <= O_MEAN_ABS, msg
     assert e["lse_max_rel"] <= LSE_REL, msg
     assert e["o_rel_l2"] <= O_REL_L2, msg
+    return e
+
+
+def assert_close_fp8(o_gpu, lse_gpu, o_ref, lse_ref, v_max: float, what: str = "") -> dict:
+    """The e4m3 bounds above; v_max = max |v| of the dequantised V."""
+    e = errors(o_gpu, lse_gpu, o_ref, lse_ref)
+    RECORDED.append({"what": what, **e})
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    msg = f"{what}: {e}"
+    assert e["finite"], msg
+    assert e["o_max_abs"] <= 2.0 ** -4 * v_max + 2.0 ** -8 * float(np.abs(o_ref).max()), msg
+    assert e["o_mean_abs"] <= FP8_O_MEAN_REL * float(np.abs(o_ref).mean()), msg
+    assert e["lse_max_rel"] <= LSE_REL, msg
+    assert e["o_rel_l2"] <= FP8_O_REL_L2, msg
     return e

@@ -164,3 +164,20 @@ def test_fwd_chunks_argument_checks(lib):
     assert _chunks(lib, d=96) == B.PA_ERR_UNSUPPORTED
     assert _chunks(lib, o=A + MB + 4096) == B.PA_ERR_INVALID_ARG         # o overlaps a K chunk
     assert _chunks(lib, Nq=0) == B.PA_OK                                 # empty query: nothing to do
+
+
+def test_fwd_fp8_argument_checks(lib):
+    f = lib.pa_attn_fwd_fp8
+    args = lambda **kw: dict(dict(q=A, k=A + MB, v=A + 2 * MB, sq=1.0, sk=1.0, sv=1.0, o=A + 3 * MB,
+                                  lse=A + 4 * MB, Nq=8, Nk=8, d=128), **kw)
+    call = lambda a: f(a["q"], a["k"], a["v"], a["sq"], a["sk"], a["sv"], a["o"], a["lse"], 1, 1, a["Nq"],
+                       a["Nk"], a["d"], 0.125, None)
+    assert call(args(q=0)) == B.PA_ERR_INVALID_ARG
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert call(args(sq=bad)) == B.PA_ERR_INVALID_ARG
+        assert call(args(sv=bad)) == B.PA_ERR_INVALID_ARG
+    assert call(args(d=64)) == B.PA_ERR_UNSUPPORTED
+    assert "d = 128" in B.last_error()
+    assert call(args(k=A + MB + 8)) == B.PA_ERR_MISALIGNED
+    assert call(args(o=A + 512)) == B.PA_ERR_INVALID_ARG          # o overlaps q (1 KB of e4m3)
+    assert call(args(Nq=0)) == B.PA_OK

@@ -17,7 +17,7 @@ import torch
 
 import oracle
 import workloads
-from tests._parity import assert_close
+from tests._parity import assert_close, assert_close_fp8
 
 pytestmark = pytest.mark.gpu
 
@@ -383,6 +383,77 @@ def test_fused_rejects_more_than_eight_chunks(pa):
     with pytest.raises(pa.PaError) as e:
         pa.attn_fwd_chunks(q, ks, [x.clone() for x in ks])
     assert e.value.code == pa.PA_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- e4m3 inputs
+
+def _quantize_e4m3(x):
+    """Per-tensor scaled e4m3: returns (x8, scale) with x ~= x8 * scale."""
+    amax = float(x.float().abs().max())
+    scale = max(amax, 1e-12) / 448.0
+    return (x.float() / scale).to(torch.float8_e4m3fn).contiguous(), scale
+
+
+def _dequant(x8, scale):
+    return x8.cpu().double() * scale
+
+
+def _fp8_check(pa, q, k, v, scale, what, rows=None):
+    (q8, sq), (k8, sk), (v8, sv) = _quantize_e4m3(q), _quantize_e4m3(k), _quantize_e4m3(v)
+    o = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full(q.shape[:3], float("nan"), device="cuda")
+    pa.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, scale=scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert pa.poll_device_status() == pa.PA_OK
+    qd, kd, vd = _dequant(q8, sq), _dequant(k8, sk), _dequant(v8, sv)
+    v_max = float(vd.abs().max())
+    if rows is None:
+        o_ref, l_ref = oracle.attention(qd, kd, vd, scale)
+        return assert_close_fp8(o, lse, o_ref, l_ref, v_max, what)
+    o_ref, l_ref = oracle.attention_rows(qd, kd, vd, scale, rows)
+    return assert_close_fp8(o[:, :, rows], lse[:, :, rows], o_ref, l_ref, v_max, what)
+
+
+def test_fp8_flux(pa):
+    w = workloads.get("flux")
+    q, k, v = workloads.make_case(w, device="cuda")
+    _fp8_check(pa, q, k, v, w.scale, "fp8 flux")
+
+
+def test_fp8_ragged_shapes(pa):
+    for (B, H, Nq, Nk) in [(1, 2, 300, 517), (2, 1, 1, 1), (1, 1, 129, 255), (1, 3, 256, 4097)]:
+        w = workloads.Workload("fp8edge", B=B, H=H, Nq=Nq, Nk=Nk, d=128, rms_qk=True, chunks=(Nk,), seed=40 + Nk)
+        q, k, v = workloads.make_case(w, device="cuda")
+        _fp8_check(pa, q, k, v, w.scale, f"fp8 edge {(B, H, Nq, Nk)}")
+
+
+def test_fp8_rising_logits(pa):
+    B, H, Nq, Nk, d = 1, 2, 200, 1100, 128
+    g = torch.Generator(device="cuda").manual_seed(79)
+    q = torch.randn((B, H, Nq, d), generator=g, device="cuda") * 0.2 + 1.0
+    ramp = torch.linspace(0.0, 1.0, Nk, device="cuda")[None, None, :, None]
+    k = torch.randn((B, H, Nk, d), generator=g, device="cuda") * 0.1 + ramp * 6.0
+    v = torch.randn((B, H, Nk, d), generator=g, device="cuda")
+    _fp8_check(pa, q, k, v, 1.0 / math.sqrt(d), "fp8 rising logits")
+
+
+def test_fp8_scales_apply(pa):
+    # the same e4m3 codes with scales (2, 0.5, 3) equal scales (1, 1, 1) on
+    # inputs multiplied out: logits unchanged, output times 3
+    w = workloads.Workload("fp8s", B=1, H=2, Nq=256, Nk=384, d=128, rms_qk=True, chunks=(384,), seed=51)
+    q, k, v = workloads.make_case(w, device="cuda")
+    (q8, _), (k8, _), (v8, _) = _quantize_e4m3(q), _quantize_e4m3(k), _quantize_e4m3(v)
+    o1, l1 = pa.attn_fwd_fp8(q8, k8, v8, 1.0, 1.0, 1.0, scale=w.scale)
+    o2, l2 = pa.attn_fwd_fp8(q8, k8, v8, 2.0, 0.5, 3.0, scale=w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(l1, l2)
+    assert (o2.float() - 3.0 * o1.float()).abs().max().item() <= 3.0 * 2 ** -7 * o1.float().abs().max().item()
+
+
+def test_fp8_rejects_bf16(pa):
+    q = torch.zeros((1, 1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(TypeError):
+        pa.attn_fwd_fp8(q, q, q, 1.0, 1.0, 1.0)
 
 
 # ---------------------------------------------------------------- CTA-pair kernel
