@@ -46,17 +46,24 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
 # kernel source whose digest is recorded with it.  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "2d699bce6e69f80019558ded24ecc2ac48f03bbf9c792d67057c5fa1b7608e43",
-    "bytes_per_launch": 84987904 + 11835648,   # dram__bytes_read.sum + dram__bytes_write.sum
+    "source_sha256": "cad86217d0aead82a2eeb65b0f63746942a1e5c870ca6749d27b2cc9699ba09a",
+    "bytes_per_launch": 84990208 + 7330560,   # dram__bytes_read.sum + dram__bytes_write.sum
     "capture": "profiles/attn_fwd_flux.md",
 }
 
 
 def _kernel_digest() -> str:
+    """SHA-256 of the forward kernel's code (comments and whitespace removed),
+    so that a recorded ncu traffic figure is used only for the code it was
+    measured on."""
+    import re
     h = hashlib.sha256()
     for f in ("ptx.cuh", "fwd_common.cuh", "attn_fwd.cuh"):
-        with open(os.path.join(ROOT, "context_blocks_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "context_blocks_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("".join(src.split()).encode())
     return h.hexdigest()
 
 

@@ -18,12 +18,18 @@
 //              loop in step, one elected lane issues)
 //   warp  9    TMA producer (Q once, then the K_j / V_j ring; same scheme)
 // Tensor memory (512 columns x 128 lanes, fp32):
-//   [0,128)        S_0 = Q_0 K_j^T   (P_0 is written back over it as bf16)
+//   [0,128)        S_0 = Q_0 K_j^T   (P_0 is written back over it: bf16
+//                  pairs, or four e4m3 per column with e4m3 inputs)
 //   [128,256)      S_1 = Q_1 K_j^T   (P_1 likewise)
 //   [256,256+D)    O_0 accumulator
 //   [256+D,256+2D) O_1 accumulator
 // Thread t of softmax warpgroup i owns TMEM lane t = query row t of tile i,
-// so row max, row sum and rescaling need no cross-thread reduction.
+// so row max, row sum and rescaling need no cross-thread reduction.  Each
+// warpgroup hands P to the MMA warp in two halves (PA_SPLIT_P), so P.V on the
+// first 64 keys starts while the second half is still being computed.
+//
+// With kFp8 the same kernel takes e4m3 Q, K, V (per-tensor scales folded into
+// the logit scale and the epilogue) and issues kind::f8f6f4 MMAs.
 //
 // Online softmax in base 2: x = s * scale * log2(e).  m_ref is the reference
 // maximum the exponentials of this row use; it moves only when a new tile's

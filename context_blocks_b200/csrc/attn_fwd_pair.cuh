@@ -19,8 +19,11 @@
 //   * the leader's tcgen05.commit arrives, by multicast, on the barrier at
 //     the same offset in both CTAs (S ready, O ready, slot free);
 //   * both CTAs' softmax warps arrive on the leader's P-ready barriers;
-//   * waits on phases another CTA completes use cluster-scope acquire, and a
-//     cluster barrier brackets set-up and teardown.
+//   * waits on phases another CTA completes go through mbar_wait_cluster
+//     (default scope unless PA_PAIR_CLUSTER_SCOPE asks for explicit cluster
+//     scope), and a cluster barrier brackets set-up and teardown.
+// The producer and MMA roles run as warp-uniform loops with one elected lane
+// issuing, as in attn_fwd.cuh.
 // The loads are plain per-CTA loads: nothing in this kernel multicasts data.
 #pragma once
 

@@ -200,8 +200,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
-// mbar_wait with cluster-scope acquire: for phases completed by the other
-// CTA of the pair (its TMA bytes, its arrivals, or the leader's commits).
+// Bounded wait for phases completed by the other CTA of the pair (its TMA
+// bytes, its arrivals, or the leader's commits); scope per
+// PA_PAIR_CLUSTER_SCOPE above.
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_word,
                                                   int* status, int code, uint64_t limit_ns) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
