@@ -67,6 +67,16 @@ def _kernel_digest() -> str:
     return h.hexdigest()
 
 
+def _workload(args):
+    """The named workload, with H replaced by --heads when given (a smaller
+    case of the same sequence shape, for profiler captures)."""
+    import dataclasses
+    w = workloads.get(args.workload)
+    if getattr(args, "heads", None):
+        w = dataclasses.replace(w, H=int(args.heads))
+    return w
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -418,7 +428,7 @@ def run_reference(args):
     ws, rank, _ = _dist_env()
     if rank != 0:
         return 0
-    w = workloads.get(args.workload)
+    w = _workload(args)
     total_budget = args.cpu_budget
     per_step = max(0.02, total_budget / max(1, args.steps + args.warmup))
     tflops_cal, t_cal, rows, desc = oracle_sample(w, per_step)
@@ -475,7 +485,7 @@ def run_ours(args):
     import context_blocks_b200 as pa
     pa.load_library()
 
-    w = workloads.get(args.workload)
+    w = _workload(args)
     peaks = _peaks()
     sampler = ClockSampler(local)
     res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier)
@@ -491,7 +501,7 @@ def run_ours(args):
     fl_launch = fl / len(w.chunks)
     achieved = fl_launch / (fwd_mean_ms * 1e-3) / 1e12
     traffic = None
-    if w.name == "flux" and NCU_TRAFFIC["source_sha256"] == _kernel_digest():
+    if w.name == "flux" and w.H == workloads.get("flux").H and NCU_TRAFFIC["source_sha256"] == _kernel_digest():
         traffic = NCU_TRAFFIC["bytes_per_launch"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
@@ -638,6 +648,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="flux", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (same sequence shape, smaller case; for profiling)")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
