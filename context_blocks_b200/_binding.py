@@ -119,7 +119,6 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=
     ``out`` / ``lse`` when given.  ``scale`` defaults to 1/sqrt(d).  With
     ``pair=True`` the CTA-pair kernel (``pa_attn_fwd_pair``, d = 128) runs.
     """
-    import torch
     _check_bf16("q", q, 4)
     _check_bf16("k", k, 4)
     _check_bf16("v", v, 4)
@@ -129,16 +128,7 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=
     Nk = k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty_like(q)
-    else:
-        _check_bf16("out", out, 4)
-        if out.shape != q.shape:
-            raise ValueError("out must have q's shape")
-    if lse is None:
-        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 [B,H,Nq] tensor")
+    out, lse = _outputs(q, out, lse)
     lib = load_library()
     fn = lib.pa_attn_fwd_pair if pair else lib.pa_attn_fwd
     rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
@@ -163,12 +153,7 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, scale:
         raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
-    else:
-        _check_bf16("out", out, 4)
-    if lse is None:
-        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    out, lse = _outputs(q, out, lse)
     rc = load_library().pa_attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
                                         float(v_scale), out.data_ptr(), lse.data_ptr(), B, H, Nq, k.shape[2], d,
                                         float(scale), _stream_handle(stream, q.device))
@@ -189,12 +174,34 @@ def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
         out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=o_parts.device)
     else:
         _check_bf16("out", out, 4)
+        if tuple(out.shape) != (B, H, N, d):
+            raise ValueError(f"out must be [B,H,N,d] = {(B, H, N, d)} (got {tuple(out.shape)})")
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=o_parts.device)
+    elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B,H,N] tensor")
     rc = load_library().pa_attn_merge(o_parts.data_ptr(), lse_parts.data_ptr(), n, out.data_ptr(),
                                       lse.data_ptr(), B, H, N, d,
                                       _stream_handle(stream, o_parts.device))
     _check(rc, "pa_attn_merge")
+    return out, lse
+
+
+def _outputs(q, out, lse):
+    """(out, lse) for a query tensor q [B,H,Nq,d]: allocated when None,
+    otherwise checked for dtype, shape and layout."""
+    import torch
+    B, H, Nq, d = q.shape
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    else:
+        _check_bf16("out", out, 4)
+        if tuple(out.shape) != (B, H, Nq, d):
+            raise ValueError("out must have q's shape")
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B,H,Nq] tensor")
     return out, lse
 
 
@@ -217,16 +224,12 @@ def _chunk_arrays(q, k_chunks, v_chunks):
 def attn_fwd_chunks(q, k_chunks, v_chunks, scale: Optional[float] = None, out=None, lse=None, stream=None):
     """Attention of q over the concatenation of the K/V chunks (up to 8) in a
     single launch (``pa_attn_fwd_chunks``); no partial results are written."""
-    import torch
     _check_bf16("q", q, 4)
     B, H, Nq, d = q.shape
     kp, vp, nk, n = _chunk_arrays(q, k_chunks, v_chunks)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    out, lse = _outputs(q, out, lse)
     rc = load_library().pa_attn_fwd_chunks(q.data_ptr(), kp, vp, nk, n, out.data_ptr(), lse.data_ptr(),
                                            B, H, Nq, d, float(scale), _stream_handle(stream, q.device))
     _check(rc, "pa_attn_fwd_chunks")
@@ -239,26 +242,12 @@ def attn_chunks_noalloc(q, k_chunks, v_chunks, scale: Optional[float] = None, ou
     its fixed static array instead of allocating them (see the header for the
     size limit and the sharing rules).  Outputs are allocated here only when
     not given."""
-    import torch
     _check_bf16("q", q, 4)
     B, H, Nq, d = q.shape
-    n = len(k_chunks)
-    if n < 1 or len(v_chunks) != n:
-        raise ValueError("need at least one chunk and as many V chunks as K chunks")
-    for kc, vc in zip(k_chunks, v_chunks):
-        _check_bf16("k chunk", kc, 4)
-        _check_bf16("v chunk", vc, 4)
-        if kc.shape != vc.shape or kc.shape[:2] != (B, H) or kc.shape[3] != d:
-            raise ValueError("chunk shapes must be [B, H, n_c, d] matching q")
+    kp, vp, nk, n = _chunk_arrays(q, k_chunks, v_chunks)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    kp = (ctypes.c_void_p * n)(*[kc.data_ptr() for kc in k_chunks])
-    vp = (ctypes.c_void_p * n)(*[vc.data_ptr() for vc in v_chunks])
-    nk = (ctypes.c_int * n)(*[kc.shape[2] for kc in k_chunks])
+    out, lse = _outputs(q, out, lse)
     rc = load_library().pa_attn_chunks_noalloc(q.data_ptr(), kp, vp, nk, n, out.data_ptr(), lse.data_ptr(),
                                                B, H, Nq, d, float(scale), _stream_handle(stream, q.device))
     _check(rc, "pa_attn_chunks_noalloc")

@@ -181,3 +181,18 @@ def test_fwd_fp8_argument_checks(lib):
     assert call(args(k=A + MB + 8)) == B.PA_ERR_MISALIGNED
     assert call(args(o=A + 512)) == B.PA_ERR_INVALID_ARG          # o overlaps q (1 KB of e4m3)
     assert call(args(Nq=0)) == B.PA_OK
+
+
+def test_output_checks_refuse_wrong_shapes(monkeypatch):
+    # The C ABI cannot see buffer sizes, so the binding refuses outputs of the
+    # wrong shape before any launch.  _check_bf16's device test is relaxed so
+    # that CPU tensors stand in for device ones here.
+    import torch
+    monkeypatch.setattr(B, "_check_bf16", lambda name, t, ndim: None)
+    q = torch.zeros((1, 2, 8, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B._outputs(q, torch.zeros((1, 2, 7, 64), dtype=torch.bfloat16), None)
+    with pytest.raises(ValueError):
+        B._outputs(q, None, torch.zeros((1, 2, 8), dtype=torch.float64))
+    o, l = B._outputs(q, None, None)
+    assert tuple(o.shape) == (1, 2, 8, 64) and tuple(l.shape) == (1, 2, 8)

@@ -450,6 +450,15 @@ def test_fp8_scales_apply(pa):
     assert (o2.float() - 3.0 * o1.float()).abs().max().item() <= 3.0 * 2 ** -7 * o1.float().abs().max().item()
 
 
+def test_merge_rejects_wrong_output_shapes(pa):
+    op = torch.zeros((2, 1, 2, 16, 64), dtype=torch.bfloat16, device="cuda")
+    lp = torch.zeros((2, 1, 2, 16), dtype=torch.float32, device="cuda")
+    with pytest.raises(ValueError):
+        pa.attn_merge(op, lp, out=torch.empty((1, 2, 8, 64), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        pa.attn_merge(op, lp, lse=torch.empty((1, 2, 8), dtype=torch.float32, device="cuda"))
+
+
 def test_fp8_rejects_bf16(pa):
     q = torch.zeros((1, 1, 8, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(TypeError):
