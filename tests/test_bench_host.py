@@ -132,3 +132,12 @@ def test_reference_arm_nonzero_rank_exits_quietly():
     r = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "3"],
                    {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_heads_override_keeps_the_sequence_shape():
+    import argparse
+    import bench
+    w = bench._workload(argparse.Namespace(workload="hunyuan", heads=4))
+    h = workloads.get("hunyuan")
+    assert (w.H, w.Nq, w.Nk, w.d, w.chunks) == (4, h.Nq, h.Nk, h.d, h.chunks)
+    assert bench._workload(argparse.Namespace(workload="flux", heads=None)) == workloads.get("flux")
