@@ -623,6 +623,28 @@ def extra_measurements(pa, device, peaks):
         out[name + "_fp8"] = {"fwd_ms_per_launch": ms, "fwd_tflops": tf,
                               "frac_of_fp8_peak": tf / (2.0 * peaks["bf16_tflops"]),
                               "peak_basis": "2 x measured bf16 burst (nominal e4m3/bf16 ratio)"}
+    # e4m3 quantisation (pa_quantize_e4m3) of a HunyuanVideo-sized Q tensor
+    # (0.73 GB bf16, far above L2): algorithmic bytes = 2 read + 1 written per
+    # element (the kernel streams x twice: amax, then convert).
+    import torch
+    h = workloads.get("hunyuan")
+    x = torch.randn((h.B * h.H * h.Nq * h.d,), device=device).to(torch.bfloat16)
+    q8 = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=device)
+    sc = torch.empty((1,), dtype=torch.float32, device=device)
+    for _ in range(3):
+        pa.quantize_e4m3(x, out=q8, scale=sc)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(10):
+        pa.quantize_e4m3(x, out=q8, scale=sc)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / 10
+    out["quantize_e4m3"] = {"elements": int(x.numel()), "ms": ms,
+                            "gbs": 3.0 * x.numel() / (ms * 1e-3) / 1e9,
+                            "frac_of_hbm": 3.0 * x.numel() / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del x, q8
     # The CTA-pair forward kernel (pa_attn_fwd_pair) on the FLUX-shaped workload.
     wf = workloads.get("flux")
     r = time_workload(pa, wf, 200, 10, device, pair=True)

@@ -31,6 +31,8 @@ SIGNATURES = {
     "pa_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_fwd_pair": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_fwd_fp8": (_I, [_VP, _VP, _VP, _F, _F, _F, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
+    "pa_attn_fwd_fp8_dev": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
+    "pa_quantize_e4m3": (_I, [_VP, ctypes.c_longlong, _VP, _VP, _VP]),
     "pa_attn_fwd_chunks": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _VP]),
     "pa_attn_chunks_noalloc": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
@@ -154,11 +156,44 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, scale:
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out, lse = _outputs(q, out, lse)
+    scales = (q_scale, k_scale, v_scale)
+    if all(isinstance(x, torch.Tensor) for x in scales):
+        # device-resident scales (as pa_quantize_e4m3 writes them)
+        for x in scales:
+            if x.dtype != torch.float32 or x.numel() != 1 or x.device != q.device:
+                raise ValueError("device scales must be one-element float32 tensors on q's device")
+        rc = load_library().pa_attn_fwd_fp8_dev(q.data_ptr(), k.data_ptr(), v.data_ptr(), *[x.data_ptr() for x in scales],
+                                                out.data_ptr(), lse.data_ptr(), B, H, Nq, k.shape[2], d, float(scale),
+                                                _stream_handle(stream, q.device))
+        _check(rc, "pa_attn_fwd_fp8_dev")
+        return out, lse
     rc = load_library().pa_attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
                                         float(v_scale), out.data_ptr(), lse.data_ptr(), B, H, Nq, k.shape[2], d,
                                         float(scale), _stream_handle(stream, q.device))
     _check(rc, "pa_attn_fwd_fp8")
     return out, lse
+
+
+def quantize_e4m3(x, out=None, scale=None, stream=None):
+    """Per-tensor e4m3 quantisation of a bf16 tensor on the device
+    (``pa_quantize_e4m3``): returns (q torch.float8_e4m3fn of x's shape,
+    scale one-element float32 device tensor) with x ~= scale * q."""
+    import torch
+    if not isinstance(x, torch.Tensor) or x.dtype != torch.bfloat16 or x.device.type != "cuda" \
+            or not x.is_contiguous():
+        raise TypeError("x must be a contiguous bfloat16 CUDA tensor")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    elif out.dtype != torch.float8_e4m3fn or out.shape != x.shape or not out.is_contiguous():
+        raise ValueError("out must be a contiguous float8_e4m3fn tensor of x's shape")
+    if scale is None:
+        scale = torch.empty((1,), dtype=torch.float32, device=x.device)
+    elif scale.dtype != torch.float32 or scale.numel() != 1:
+        raise ValueError("scale must be a one-element float32 tensor")
+    rc = load_library().pa_quantize_e4m3(x.data_ptr(), x.numel(), out.data_ptr(), scale.data_ptr(),
+                                         _stream_handle(stream, x.device))
+    _check(rc, "pa_quantize_e4m3")
+    return out, scale
 
 
 def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):

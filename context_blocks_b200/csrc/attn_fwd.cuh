@@ -378,7 +378,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tS = tmem + i * kBN + lane_off;
     const uint32_t tO = tmem + 2 * kBN + i * D + lane_off;
     const int row = q0 + i * kBM + t;
-    const float c = p.scale_log2;
+    // Logit scale in log2 units; e4m3 inputs may carry their dequantisation
+    // scales in device memory.
+    float c = p.scale_log2;
+    if constexpr (kFp8) c *= (p.dscale_q != nullptr) ? __ldg(p.dscale_q) * __ldg(p.dscale_k) : p.qk_scale;
     float m_ref = -INFINITY;
     float l = 0.f;
     bool ok = true;
@@ -523,7 +526,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      const float inv_l = p.o_scale / l;
+      float inv_l = 1.f / l;
+      if constexpr (kFp8) inv_l = ((p.dscale_v != nullptr) ? __ldg(p.dscale_v) : p.o_scale) / l;
       const bool in_range = row < p.Nq;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.Nq + row) * D;
 #pragma unroll

@@ -30,7 +30,13 @@ struct FwdParams {
   float scale_log2;     // scale * log2(e)
   int* status;          // device status word
   unsigned long long timeout_ns;
+  float qk_scale;       // logits are also multiplied by this (q_scale * k_scale; 1 for bf16)
   float o_scale;        // O is multiplied by this (the V dequantisation scale; 1 for bf16)
+  // Device-side dequantisation scales (e4m3 inputs), used instead of
+  // qk_scale / o_scale when dscale_q is not null.
+  const float* dscale_q;
+  const float* dscale_k;
+  const float* dscale_v;
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {

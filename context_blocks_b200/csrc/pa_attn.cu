@@ -12,6 +12,7 @@
 
 #include "attn_fwd.cuh"
 #include "attn_fwd_pair.cuh"
+#include "quantize.cuh"
 #include "fwd_common.cuh"
 #include "lse_merge.cuh"
 #include "pa_attn.h"
@@ -173,7 +174,7 @@ int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int
 template <int D, bool kFp8 = false>
 int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void* const* v, const int* nk,
                int n_chunks, void* o, float* lse, int BH, int Nq, float scale, cudaStream_t stream,
-               float qk_scale = 1.f, float o_scale = 1.f) {
+               float qk_scale = 1.f, float o_scale = 1.f, const float* const* dscales = nullptr) {
   using L = pa::single::FwdLayout<D, kFp8>;
   CUtensorMap tq;
   pa::single::KvChunks kv;
@@ -212,10 +213,14 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   prm.Nq = Nq;
   prm.Nk = static_cast<int>(nk_total);
   prm.n_kv_tiles = static_cast<int>(tiles_total);
-  prm.scale_log2 = scale * qk_scale * 1.4426950408889634f;
+  prm.scale_log2 = scale * 1.4426950408889634f;
   prm.status = st->status;
   prm.timeout_ns = kDefaultTimeoutNs;
+  prm.qk_scale = qk_scale;
   prm.o_scale = o_scale;
+  prm.dscale_q = dscales ? dscales[0] : nullptr;
+  prm.dscale_k = dscales ? dscales[1] : nullptr;
+  prm.dscale_v = dscales ? dscales[2] : nullptr;
   dim3 grid((Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM), BH);
   kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, kv, prm);
   cudaError_t e = cudaGetLastError();
@@ -258,7 +263,9 @@ int launch_fwd_pair(DeviceState* st, const void* q, const void* k, const void* v
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.status = st->status;
   prm.timeout_ns = kDefaultTimeoutNs;
+  prm.qk_scale = 1.f;
   prm.o_scale = 1.f;
+  prm.dscale_q = prm.dscale_k = prm.dscale_v = nullptr;
   const int rows_per_pair = 2 * pa::kQTiles * pa::kBM;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ((Nq + rows_per_pair - 1) / rows_per_pair), BH);
@@ -364,6 +371,60 @@ int pa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, 
   if (rc != PA_OK || st == nullptr) return rc;
   return launch_fwd<128, true>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, static_cast<cudaStream_t>(stream),
                                q_scale * k_scale, v_scale);
+}
+
+int pa_attn_fwd_fp8_dev(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
+                        const float* v_scale, void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
+                        void* stream) {
+  g_err[0] = '\0';
+  if (!q_scale || !k_scale || !v_scale) return fail(PA_ERR_INVALID_ARG, "null scale pointer");
+  if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
+    return fail(PA_ERR_MISALIGNED, "scale pointers must be 4-byte aligned");
+  DeviceState* st = nullptr;
+  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, true, 1);  // host-side checks
+  if (rc != PA_OK) return rc;
+  if (d != 128) return fail(PA_ERR_UNSUPPORTED, "the e4m3 forward needs d = 128 (got %d)", d);
+  rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, false, 1);
+  if (rc != PA_OK || st == nullptr) return rc;
+  int dev = 0;
+  const float* sp[3] = {q_scale, k_scale, v_scale};
+  for (int i = 0; i < 3; ++i)
+    if ((rc = check_device_ptr(sp[i], "scale", &dev)) != PA_OK) return rc;
+  return launch_fwd<128, true>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, static_cast<cudaStream_t>(stream),
+                               1.f, 1.f, sp);
+}
+
+int pa_quantize_e4m3(const void* x, long long n, void* q, float* scale, void* stream) {
+  g_err[0] = '\0';
+  if (!x || !q || !scale) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (n < 1) return fail(PA_ERR_INVALID_ARG, "n must be >= 1 (got %lld)", n);
+  if (!aligned(x, 16) || !aligned(q, 16)) return fail(PA_ERR_MISALIGNED, "x and q must be 16-byte aligned");
+  if (!aligned(scale, 4)) return fail(PA_ERR_MISALIGNED, "scale must be 4-byte aligned");
+  if (overlap(x, static_cast<uint64_t>(n) * 2, q, static_cast<uint64_t>(n)) ||
+      overlap(x, static_cast<uint64_t>(n) * 2, scale, 4) || overlap(q, static_cast<uint64_t>(n), scale, 4))
+    return fail(PA_ERR_INVALID_ARG, "x, q and scale must not overlap");
+  (void)cudaGetLastError();
+  int dev = 0, rc;
+  const void* ptrs[3] = {x, q, scale};
+  const char* names[3] = {"x", "q", "scale"};
+  for (int i = 0; i < 3; ++i)
+    if ((rc = check_device_ptr(ptrs[i], names[i], &dev)) != PA_OK) return rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(dev, &st)) != PA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned* word = reinterpret_cast<unsigned*>(scale);
+  cudaError_t e = cudaMemsetAsync(word, 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  const long long n8 = n / 8;
+  const long long want = (n8 + pa::quant::kThreads - 1) / pa::quant::kThreads;
+  const int grid = static_cast<int>(std::max(1LL, std::min(want, 8LL * st->sm_count)));
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  pa::quant::amax_kernel<<<grid, pa::quant::kThreads, 0, s>>>(xb, n, word);
+  pa::quant::quantize_kernel<<<grid, pa::quant::kThreads, 0, s>>>(xb, n, word, static_cast<uint8_t*>(q));
+  pa::quant::scale_kernel<<<1, 1, 0, s>>>(word);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return PA_OK;
 }
 
 int pa_attn_fwd_chunks(const void* q, const void* const* k_chunks, const void* const* v_chunks,

@@ -108,6 +108,47 @@ int pa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, 
                     float scale, void* stream);
 
 /*
+ * pa_attn_fwd_fp8_dev - pa_attn_fwd_fp8 with the three dequantisation scales
+ * read from device memory (each a float, e.g. written by pa_quantize_e4m3),
+ * so that quantising and attending need no host synchronisation.
+ *
+ * q_scale, k_scale, v_scale   device pointers to one float each, 4-byte aligned,
+ *                             finite and > 0 when the kernel runs (not checked:
+ *                             they are read on the device)
+ * everything else             as pa_attn_fwd_fp8
+ *
+ * Errors: as pa_attn_fwd_fp8; PA_ERR_INVALID_ARG for a null or host scale
+ * pointer, PA_ERR_MISALIGNED for a misaligned one.
+ */
+int pa_attn_fwd_fp8_dev(const void* q, const void* k, const void* v, const float* q_scale,
+                        const float* k_scale, const float* v_scale, void* o, float* lse, int B, int H,
+                        int Nq, int Nk, int d, float scale, void* stream);
+
+/*
+ * pa_quantize_e4m3 - per-tensor e4m3 quantisation of a bf16 tensor.
+ *
+ *     amax  = max_i |x[i]|
+ *     scale = amax / 448 in fp32 (1 if amax = 0)
+ *     q[i]  = e4m3 nearest to x[i] / scale (fp32 division), ties to even,
+ *             saturated to +-448                 (OCP E4M3FN codes)
+ * so that x ~= scale * decode(q); *scale is written on the device.  This is
+ * the dynamic per-tensor fp8 quantisation the pages apply to activations
+ * (diffusers "ParaAttention" guide, fp8 section), as input to
+ * pa_attn_fwd_fp8_dev.
+ *
+ * x      n bf16 values, device, 16-byte aligned             (input)
+ * q      n bytes, device, 16-byte aligned                    (output)
+ * scale  one float, device, 4-byte aligned                   (output; also
+ *        used as the reduction word while the call runs)
+ * n      >= 1
+ *
+ * Errors: PA_ERR_INVALID_ARG (null, n < 1, overlapping buffers, host memory),
+ * PA_ERR_MISALIGNED, PA_ERR_CUDA.  Three kernels and one memset are enqueued
+ * on `stream`; nothing is allocated.
+ */
+int pa_quantize_e4m3(const void* x, long long n, void* q, float* scale, void* stream);
+
+/*
  * pa_attn_fwd_chunks - attention of Q over several K/V chunks in one launch.
  *
  * The local loop of Ring Attention fused (diffusers "Context parallelism",

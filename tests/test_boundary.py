@@ -196,3 +196,19 @@ def test_output_checks_refuse_wrong_shapes(monkeypatch):
         B._outputs(q, None, torch.zeros((1, 2, 8), dtype=torch.float64))
     o, l = B._outputs(q, None, None)
     assert tuple(o.shape) == (1, 2, 8, 64) and tuple(l.shape) == (1, 2, 8)
+
+
+def test_quantize_and_fp8_dev_argument_checks(lib):
+    qz = lib.pa_quantize_e4m3
+    assert qz(0, 16, A + MB, A + 2 * MB, None) == B.PA_ERR_INVALID_ARG
+    assert qz(A, 0, A + MB, A + 2 * MB, None) == B.PA_ERR_INVALID_ARG
+    assert qz(A + 8, 16, A + MB, A + 2 * MB, None) == B.PA_ERR_MISALIGNED
+    assert qz(A, 16, A + MB, A + 2 * MB + 2, None) == B.PA_ERR_MISALIGNED
+    assert qz(A, 1024, A + 1024, A + 2 * MB, None) == B.PA_ERR_INVALID_ARG     # q overlaps x (2 KB)
+    f = lib.pa_attn_fwd_fp8_dev
+    ok = dict(q=A, k=A + MB, v=A + 2 * MB, sq=A + 5 * MB, sk=A + 5 * MB + 4, sv=A + 5 * MB + 8)
+    call = lambda **kw: f(*[dict(ok, **kw)[n] for n in ("q", "k", "v", "sq", "sk", "sv")], A + 3 * MB, A + 4 * MB,
+                          1, 1, 8, 8, kw.get("d", 128), 0.125, None)
+    assert call(sk=0) == B.PA_ERR_INVALID_ARG
+    assert call(sv=A + 5 * MB + 9) == B.PA_ERR_MISALIGNED
+    assert call(d=64) == B.PA_ERR_UNSUPPORTED

@@ -422,3 +422,50 @@ def test_pins_catch_planted_merge_mistakes(kind):
 def test_unmutated_oracle_passes_every_pin():
     results = _run_pins(oracle.attention, oracle.merge)
     assert all(results.values()), results
+
+
+# ---------------------------------------------------------------- e4m3 rounding
+
+from oracle import e4m3 as E
+
+
+def test_e4m3_decode_table_fixed_points():
+    t = E.decode_table()
+    assert t[0x00] == 0.0 and t[0x38] == 1.0 and t[0x40] == 2.0 and t[0x30] == 0.5
+    assert t[0x7E] == 448.0 and t[0xFE] == -448.0
+    assert t[0x01] == 2.0 ** -9 and t[0x08] == 2.0 ** -6 and t[0x07] == 7 * 2.0 ** -9
+    assert np.isnan(t[0x7F]) and np.isnan(t[0xFF])
+    pos = t[:0x7F]
+    assert np.all(np.diff(pos) > 0)                       # codes 0..0x7E increase
+    assert np.array_equal(t[0x80:0xFF], -pos)             # sign bit
+
+
+def test_e4m3_encode_round_trip_and_ties():
+    t = E.decode_table()
+    finite = np.array([c for c in range(256) if not np.isnan(t[c])])
+    # every finite value encodes to itself (0.0 and -0.0 keep their signs)
+    for c in finite:
+        assert E.encode_rne(t[c]) == c, hex(c)
+    # midpoints go to the even code: between 1.0 (0x38) and 1.125 (0x39) -> 0x38;
+    # between 1.125 (0x39) and 1.25 (0x3A) -> 0x3A
+    assert E.encode_rne(1.0625) == 0x38 and E.encode_rne(1.1875) == 0x3A
+    # just off the midpoint goes to the nearer code
+    assert E.encode_rne(np.nextafter(1.0625, 2.0)) == 0x39
+    # saturation and the subnormal range
+    assert E.encode_rne(1e6) == 0x7E and E.encode_rne(-1e6) == 0xFE and E.encode_rne(449.0) == 0x7E
+    assert E.encode_rne(2.0 ** -10) == 0x00                  # halfway 0 .. 2^-9 -> even (0)
+    assert E.encode_rne(3 * 2.0 ** -10) == 0x02              # halfway 2^-9 .. 2^-8 -> even (0x02)
+
+
+def test_e4m3_quantize_matches_torch_cast():
+    # an independent implementation of the same rounding (PyTorch's cast)
+    import torch
+    rng = np.random.default_rng(3)
+    x = torch.from_numpy(rng.standard_normal(5000).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    codes, scale = E.quantize(x)
+    y = (x / scale).astype(np.float32)
+    ok = np.abs(y) < 448.0                                   # torch's cast does not saturate
+    tc = torch.from_numpy(y[ok]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes[ok], tc)
+    assert scale == np.float32(np.max(np.abs(x)) / np.float32(448.0))
+    assert E.quantize(np.zeros(7))[1] == 1.0 and not np.any(E.quantize(np.zeros(7))[0])

@@ -459,6 +459,41 @@ def test_merge_rejects_wrong_output_shapes(pa):
         pa.attn_merge(op, lp, lse=torch.empty((1, 2, 8), dtype=torch.float32, device="cuda"))
 
 
+def test_quantize_e4m3_bit_exact(pa):
+    from oracle import e4m3 as E
+    g = torch.Generator(device="cuda").manual_seed(61)
+    for n in (1, 7, 8, 1000, 4099, 1 << 20):
+        x = (torch.randn((n,), generator=g, device="cuda") * 3.0).to(torch.bfloat16)
+        q8, sc = pa.quantize_e4m3(x)
+        torch.cuda.synchronize()
+        xs = x.float().cpu().numpy()
+        s = np.float32(sc.item())
+        # the scale is amax / 448 in fp32; the codes are the oracle's rounding of x / s
+        assert s == np.float32(np.max(np.abs(xs)) / np.float32(448.0)), n
+        ref = E.encode_rne((xs / s).astype(np.float32))
+        got = q8.view(torch.uint8).cpu().numpy()
+        assert np.array_equal(got, ref), (n, int(np.sum(got != ref)))
+    z = torch.zeros((40,), dtype=torch.bfloat16, device="cuda")
+    q8, sc = pa.quantize_e4m3(z)
+    torch.cuda.synchronize()
+    assert sc.item() == 1.0 and not q8.view(torch.uint8).any()
+
+
+def test_fp8_device_scales_pipeline(pa):
+    # bf16 -> pa_quantize_e4m3 -> pa_attn_fwd_fp8_dev, checked against the oracle
+    # on the dequantised codes, and equal to the host-scale entry point.
+    w = workloads.Workload("fp8dev", B=1, H=3, Nq=700, Nk=1300, d=128, rms_qk=True, chunks=(1300,), seed=62)
+    q, k, v = workloads.make_case(w, device="cuda")
+    (q8, sq), (k8, sk), (v8, sv) = pa.quantize_e4m3(q), pa.quantize_e4m3(k), pa.quantize_e4m3(v)
+    o, lse = pa.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, scale=w.scale)
+    o2, l2 = pa.attn_fwd_fp8(q8, k8, v8, sq.item(), sk.item(), sv.item(), scale=w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+    qd, kd, vd = (_dequant(a, float(b.item())) for a, b in ((q8, sq), (k8, sk), (v8, sv)))
+    o_ref, l_ref = oracle.attention(qd, kd, vd, w.scale)
+    assert_close_fp8(o, lse, o_ref, l_ref, float(vd.abs().max()), "fp8 device-scale pipeline")
+
+
 def test_fp8_rejects_bf16(pa):
     q = torch.zeros((1, 1, 8, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(TypeError):
