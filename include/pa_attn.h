@@ -1,13 +1,19 @@
 /*
  * pa_attn.h - blockwise (ring-step) attention for NVIDIA B200 (sm_100a).
  *
- * A C ABI over two CUDA kernels:
+ * A C ABI whose two core entry points are:
  *
  *   pa_attn_fwd    attention of every query row against ONE key/value chunk,
  *                  returning the normalised partial output O and the natural
  *                  log-sum-exp LSE of the scaled logits over that chunk;
  *   pa_attn_merge  the exact combination of n such partial results, computed
  *                  over disjoint key chunks, into the full-sequence result.
+ *
+ * Around them: pa_attn_fwd_chunks (up to 8 chunks in one launch, no
+ * partials), pa_attn_fwd_pair (the same forward on CTA pairs),
+ * pa_attn_fwd_fp8 / pa_attn_fwd_fp8_dev with pa_quantize_e4m3 (e4m3 inputs),
+ * pa_attn_chunks_noalloc (chunks + merge with library-owned static scratch),
+ * and the status helpers at the end of this file.
  *
  * Together they are the per-device step of Ring Attention as the diffusers
  * guide "Context parallelism" describes it (section "Ring Attention": each
@@ -24,13 +30,14 @@
  * ---------------------------------------
  * - Layouts are contiguous, row-major, head dimension innermost:
  *     q, o   [B, H, Nq, d] bf16          k, v   [B, H, Nk, d] bf16
+ *     (q, k, v are one-byte e4m3 codes in the fp8 entry points; o stays bf16)
  *     lse    [B, H, Nq]    fp32, natural log
  * - All tensor pointers are DEVICE pointers on the current CUDA device, owned
  *   and allocated by the caller.  The library allocates no memory in any call.
  *   Inputs and outputs must not overlap.
  * - q, k, v, o and o_parts must be 16-byte aligned (TMA / vector access);
  *   lse and lse_parts 4-byte aligned.
- * - d must be 64 or 128.
+ * - d must be 64 or 128 (128 for the CTA-pair and e4m3 entry points).
  * - `stream` is a cudaStream_t (0 = legacy default stream).  Calls are fully
  *   asynchronous: they validate arguments on the host, enqueue kernels on
  *   `stream` and return.  They never synchronise the host and never copy
