@@ -46,8 +46,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
 # kernel source whose digest is recorded with it.  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "cad86217d0aead82a2eeb65b0f63746942a1e5c870ca6749d27b2cc9699ba09a",
-    "bytes_per_launch": 84990208 + 7330560,   # dram__bytes_read.sum + dram__bytes_write.sum
+    "source_sha256": "c04f091c8d0496fe9c6bf43b9be3785dd74a359bc103c5c2b6d94497361b1e65",
+    "bytes_per_launch": 84987392 + 5752576,   # dram__bytes_read.sum + dram__bytes_write.sum
     "capture": "profiles/attn_fwd_flux.md",
 }
 
