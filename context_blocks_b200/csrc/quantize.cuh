@@ -2,8 +2,9 @@
 // forward (the storage format the diffusers "ParaAttention" guide quantises
 // activations to, its fp8 section):
 //     amax  = max |x|
-//     scale = amax / 448 in fp32 (1 when amax = 0)
-//     q     = e4m3 nearest to x / scale (fp32 IEEE division), ties to even,
+//     scale = amax / 448 in fp32 (1 when amax = 0)          (dequantisation)
+//     inv   = 448 / amax in fp32 (1 when amax = 0)          (quantisation)
+//     q     = e4m3 nearest to x * inv (one fp32 multiply), ties to even,
 //             saturated to +-448
 // Three stream-ordered launches share the caller's 4-byte `scale` word:
 //   1. amax_kernel: |x| as bf16 bits (non-negative, so integer order is value
@@ -35,7 +36,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __nv_bfloat16* __r
   uint32_t m = 0;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
-    const uint4 v = __ldcs(x8 + i);
+    const uint4 v = __ldg(x8 + i);  // cached: a tensor that fits in L2 is read from there by the second pass
     m = max(m, max(max(abs_bits2(v.x), abs_bits2(v.y)), max(abs_bits2(v.z), abs_bits2(v.w))));
   }
   if (blockIdx.x == 0 && threadIdx.x < n - n8 * 8) {
@@ -51,30 +52,35 @@ __device__ __forceinline__ float scale_from_word(unsigned w) {
   const float amax = __uint_as_float(w << 16);  // bf16 bits -> fp32
   return amax / 448.f;
 }
+__device__ __forceinline__ float inv_from_word(unsigned w) {
+  if (w == 0) return 1.f;
+  return 448.f / __uint_as_float(w << 16);
+}
 
-__device__ __forceinline__ uint32_t quant4(uint32_t a, uint32_t b, float s) {
+__device__ __forceinline__ uint32_t quant4(uint32_t a, uint32_t b, float inv) {
   // two bf16 pairs -> four e4m3 bytes (lowest element in the low byte)
   const float x0 = __uint_as_float(a << 16), x1 = __uint_as_float(a & 0xFFFF0000u);
   const float x2 = __uint_as_float(b << 16), x3 = __uint_as_float(b & 0xFFFF0000u);
-  return pack_e4m3x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s)) | (pack_e4m3x2(__fdiv_rn(x2, s), __fdiv_rn(x3, s)) << 16);
+  return pack_e4m3x2(__fmul_rn(x0, inv), __fmul_rn(x1, inv)) |
+         (pack_e4m3x2(__fmul_rn(x2, inv), __fmul_rn(x3, inv)) << 16);
 }
 
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const __nv_bfloat16* __restrict__ x, long long n,
                                                             const unsigned* __restrict__ word,
                                                             uint8_t* __restrict__ q) {
-  const float s = scale_from_word(*word);
+  const float inv = inv_from_word(*word);
   const long long n8 = n / 8;
   const uint4* x8 = reinterpret_cast<const uint4*>(x);
   uint2* q8 = reinterpret_cast<uint2*>(q);
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
     const uint4 v = __ldcs(x8 + i);
-    q8[i] = make_uint2(quant4(v.x, v.y, s), quant4(v.z, v.w, s));
+    q8[i] = make_uint2(quant4(v.x, v.y, inv), quant4(v.z, v.w, inv));
   }
   if (blockIdx.x == 0 && threadIdx.x < n - n8 * 8) {
     const long long e = n8 * 8 + threadIdx.x;
     const float xv = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(x)[e]) << 16);
-    q[e] = static_cast<uint8_t>(pack_e4m3x2(__fdiv_rn(xv, s), 0.f) & 0xFFu);
+    q[e] = static_cast<uint8_t>(pack_e4m3x2(__fmul_rn(xv, inv), 0.f) & 0xFFu);
   }
 }
 

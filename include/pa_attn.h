@@ -135,8 +135,9 @@ int pa_attn_fwd_fp8_dev(const void* q, const void* k, const void* v, const float
  * pa_quantize_e4m3 - per-tensor e4m3 quantisation of a bf16 tensor.
  *
  *     amax  = max_i |x[i]|
- *     scale = amax / 448 in fp32 (1 if amax = 0)
- *     q[i]  = e4m3 nearest to x[i] / scale (fp32 division), ties to even,
+ *     scale = amax / 448 in fp32 (1 if amax = 0)     (written to *scale)
+ *     inv   = 448 / amax in fp32 (1 if amax = 0)
+ *     q[i]  = e4m3 nearest to x[i] * inv (fp32 multiply), ties to even,
  *             saturated to +-448                 (OCP E4M3FN codes)
  * so that x ~= scale * decode(q); *scale is written on the device.  This is
  * the dynamic per-tensor fp8 quantisation the pages apply to activations

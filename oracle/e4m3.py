@@ -15,7 +15,8 @@ Quantisation as the library does it (the plain per-tensor reading):
 
     amax  = max |x|                      (x as given, bf16 values)
     scale = amax / 448   in float32      (scale = 1 when amax = 0)
-    y     = x / scale    in float32      (IEEE division)
+    inv   = 448 / amax   in float32      (inv = 1 when amax = 0)
+    y     = x * inv      in float32      (one multiply per element)
     code  = e4m3 nearest to y, ties to the even code, saturated to +-448
 
 so that x ~= scale * decode(code).
@@ -71,5 +72,6 @@ def quantize(x) -> tuple:
     x32 = np.asarray(x, dtype=np.float32)
     amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0)
     scale = np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(E4M3_MAX))
-    y = (x32 / scale).astype(np.float32)
+    inv = np.float32(1.0) if amax == 0 else np.float32(np.float32(E4M3_MAX) / amax)
+    y = (x32 * inv).astype(np.float32)
     return encode_rne(y), scale

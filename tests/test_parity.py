@@ -468,9 +468,9 @@ def test_quantize_e4m3_bit_exact(pa):
         torch.cuda.synchronize()
         xs = x.float().cpu().numpy()
         s = np.float32(sc.item())
-        # the scale is amax / 448 in fp32; the codes are the oracle's rounding of x / s
-        assert s == np.float32(np.max(np.abs(xs)) / np.float32(448.0)), n
-        ref = E.encode_rne((xs / s).astype(np.float32))
+        # the scale is amax / 448 in fp32; the codes are the oracle's quantisation
+        ref, s_ref = E.quantize(xs)
+        assert s == s_ref, n
         got = q8.view(torch.uint8).cpu().numpy()
         assert np.array_equal(got, ref), (n, int(np.sum(got != ref)))
     z = torch.zeros((40,), dtype=torch.bfloat16, device="cuda")
