@@ -187,14 +187,26 @@ def aggregate_throughput(flops_per_step_per_rank: float, steps: int, world: int,
 class Step:
     """Buffers and launches of one hot-path step on one workload."""
 
-    def __init__(self, w: workloads.Workload, sets: int, device, pair: bool = False):
+    def __init__(self, w: workloads.Workload, sets: int, device, pair: bool = False, fp8: bool = False, pa=None):
         import torch
         self.w = w
         self.pair = pair
+        self.fp8 = fp8
         self.sets = []
         n = len(w.chunks)
+        if fp8 and n != 1:
+            raise SystemExit("--fp8 times the single-chunk e4m3 forward: pick a one-chunk workload")
         for s in range(sets):
             q, k, v = workloads.make_case(w, device=device, seed=w.seed + 1000 * s)
+            if fp8:
+                # per-tensor e4m3 inputs made by the library's own quantiser
+                # (outside the timed region), scales left in device memory
+                qs, ks, vs = pa.quantize_e4m3(q), pa.quantize_e4m3(k), pa.quantize_e4m3(v)
+                o = torch.empty_like(q)
+                lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+                self.sets.append((qs, [(ks, vs)], o, lse, None, None))
+                del q, k, v
+                continue
             pairs = workloads.split_keys(k, v, w.chunks)
             del k, v
             o = torch.empty_like(q)
@@ -208,6 +220,10 @@ class Step:
 
     def bytes_resident(self) -> int:
         tot = 0
+        if self.fp8:
+            for (q8, _), [((k8, _), (v8, _))], o, lse, _, _ in self.sets:
+                tot += q8.numel() + k8.numel() + v8.numel() + o.numel() * 2 + lse.numel() * 4
+            return tot
         for q, pairs, o, lse, op, lp in self.sets:
             tot += q.numel() * 2 + sum(k.numel() * 4 for k, _ in pairs) + o.numel() * 2 + lse.numel() * 4
             if op is not None:
@@ -215,6 +231,14 @@ class Step:
         return tot
 
     def run(self, i: int, pa, fwd_events=None, merge_events=None):
+        if self.fp8:
+            (q8, sq), [((k8, sk), (v8, sv))], o, lse, _, _ = self.sets[i % len(self.sets)]
+            if fwd_events is not None:
+                fwd_events[0].append(_record())
+            pa.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, scale=self.w.scale, out=o, lse=lse)
+            if fwd_events is not None:
+                fwd_events[1].append(_record())
+            return
         q, pairs, o, lse, o_parts, lse_parts = self.sets[i % len(self.sets)]
         n = len(pairs)
         for p, (k, v) in enumerate(pairs):
@@ -240,16 +264,18 @@ def _record():
     return e
 
 
-def _sets_for(w: workloads.Workload) -> int:
+def _sets_for(w: workloads.Workload, fp8: bool = False) -> int:
     per_set = workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk, w.d)
+    if fp8:  # Q, K, V at one byte per element
+        per_set -= (w.Nq + 2 * w.Nk) * w.d * w.B * w.H
     return max(1, min(8, math.ceil(2.5 * L2_BYTES / per_set)))
 
 
-def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, pair=False):
+def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, pair=False, fp8=False):
     """Device time of `steps` steps (CUDA events on the launching stream,
     synchronised on both sides).  Returns a dict of timings."""
     import torch
-    st = Step(w, _sets_for(w), device, pair=pair)
+    st = Step(w, _sets_for(w, fp8), device, pair=pair, fp8=fp8, pa=pa)
     for i in range(warmup):
         st.run(i, pa)
     torch.cuda.synchronize()
@@ -288,7 +314,7 @@ class _Null:
         return False
 
 
-def e2e_throughput(pa, w, steps, device):
+def e2e_throughput(pa, w, steps, device, fp8: bool = False):
     """Same metric through the public API from pinned HOST buffers: every
     step copies q and the K/V chunks host->device, runs the step, and copies
     o and lse device->host; all inside the timed region.
@@ -297,44 +323,52 @@ def e2e_throughput(pa, w, steps, device):
     output buffers, so one step's host->device copy overlaps the previous
     step's attention and device->host copy (the copy engines of the two
     directions and the SMs work at the same time).  Each step still moves
-    all of its own bytes."""
+    all of its own bytes.  With fp8 the host holds e4m3 codes (quantised once
+    by the library, scales kept on the device) and each step uploads those."""
     import torch
     q, k, v = workloads.make_case(w, device=device)
-    pairs = workloads.split_keys(k, v, w.chunks)
-    hq = q.cpu().pin_memory()
-    hpairs = [(kk.cpu().pin_memory(), vv.cpu().pin_memory()) for kk, vv in pairs]
-    n = len(pairs)
     B, H, Nq, d = q.shape
-    del k, v, pairs
+    if fp8:
+        quant = [pa.quantize_e4m3(x) for x in (q, k, v)]
+        host_in = [x8.view(torch.uint8).cpu().pin_memory() for x8, _ in quant]
+        scales = [sc for _, sc in quant]
+        del quant
+    else:
+        pairs = workloads.split_keys(k, v, w.chunks)
+        host_in = [q.cpu().pin_memory()] + [t.cpu().pin_memory() for pr in pairs for t in pr]
+        del pairs
+    n = len(w.chunks)
+    del k, v
 
     class Lane:
         def __init__(self):
             self.stream = torch.cuda.Stream(device=device)
-            self.dq = torch.empty_like(q)
-            self.dpairs = [(torch.empty(hk.shape, dtype=hk.dtype, device=device),
-                            torch.empty(hv.shape, dtype=hv.dtype, device=device)) for hk, hv in hpairs]
+            self.dev_in = [torch.empty(h.shape, dtype=h.dtype, device=device) for h in host_in]
             self.o_parts = torch.empty((n, B, H, Nq, d), dtype=torch.bfloat16, device=device) if n > 1 else None
             self.lse_parts = torch.empty((n, B, H, Nq), dtype=torch.float32, device=device) if n > 1 else None
-            self.o = torch.empty_like(q)
+            self.o = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=device)
             self.lse = torch.empty((B, H, Nq), dtype=torch.float32, device=device)
             self.ho = torch.empty(self.o.shape, dtype=self.o.dtype, pin_memory=True)
             self.hl = torch.empty(self.lse.shape, dtype=self.lse.dtype, pin_memory=True)
 
         def step(self):
             with torch.cuda.stream(self.stream):
-                self.dq.copy_(hq, non_blocking=True)
-                for (dk, dv), (hk, hv) in zip(self.dpairs, hpairs):
-                    dk.copy_(hk, non_blocking=True)
+                for dv, hv in zip(self.dev_in, host_in):
                     dv.copy_(hv, non_blocking=True)
-                pa.blockwise_attention(self.dq, [a for a, _ in self.dpairs], [b for _, b in self.dpairs],
-                                       scale=w.scale, o_parts=self.o_parts, lse_parts=self.lse_parts,
-                                       out=self.o, lse=self.lse, stream=self.stream)
+                if fp8:
+                    q8, k8, v8 = (t.view(torch.float8_e4m3fn) for t in self.dev_in)
+                    pa.attn_fwd_fp8(q8, k8, v8, *scales, scale=w.scale, out=self.o, lse=self.lse,
+                                    stream=self.stream)
+                else:
+                    dq, rest = self.dev_in[0], self.dev_in[1:]
+                    pa.blockwise_attention(dq, rest[0::2], rest[1::2], scale=w.scale, o_parts=self.o_parts,
+                                           lse_parts=self.lse_parts, out=self.o, lse=self.lse, stream=self.stream)
                 self.ho.copy_(self.o, non_blocking=True)
                 self.hl.copy_(self.lse, non_blocking=True)
 
     lanes = [Lane(), Lane()]
     del q
-    h2d = hq.numel() * 2 + sum(a.numel() * 2 + b.numel() * 2 for a, b in hpairs)
+    h2d = sum(h.numel() * h.element_size() for h in host_in)
     d2h = lanes[0].ho.numel() * 2 + lanes[0].hl.numel() * 4
 
     for i in range(2):
@@ -488,7 +522,8 @@ def run_ours(args):
     w = _workload(args)
     peaks = _peaks()
     sampler = ClockSampler(local)
-    res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier)
+    fp8 = bool(getattr(args, "fp8", False))
+    res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier, fp8=fp8)
     if res["status"] != 0:
         raise SystemExit(f"device status {res['status']} after the timed region")
     max_ms = max_over_ranks(res["total_ms"], device)
@@ -501,18 +536,25 @@ def run_ours(args):
     fl_launch = fl / len(w.chunks)
     achieved = fl_launch / (fwd_mean_ms * 1e-3) / 1e12
     traffic = None
-    if w.name == "flux" and w.H == workloads.get("flux").H and NCU_TRAFFIC["source_sha256"] == _kernel_digest():
+    if (not fp8 and w.name == "flux" and w.H == workloads.get("flux").H
+            and NCU_TRAFFIC["source_sha256"] == _kernel_digest()):
         traffic = NCU_TRAFFIC["bytes_per_launch"]
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-            "kernel": "attn_fwd_kernel<128>", "launch_ms": fwd_mean_ms,
-            "peak_basis": f"{peaks['source']} burst bf16 (MEASURED_PEAKS.json bf16_tflops); "
-                          f"frac of sustained {achieved / peaks['bf16_tflops_sustained']:.3f}",
-            "algorithmic_bytes_per_launch": workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk // len(w.chunks), w.d)}
+    # e4m3 contractions: the measured bf16 peak times the nominal e4m3/bf16 ratio of 2
+    peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+    alg_bytes = workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk // len(w.chunks), w.d)
+    if fp8:
+        alg_bytes -= (w.Nq + 2 * (w.Nk // len(w.chunks))) * w.d * w.B * w.H
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic,
+            "kernel": f"attn_fwd_kernel<{w.d}, {'true' if fp8 else 'false'}>", "launch_ms": fwd_mean_ms,
+            "peak_basis": (f"{peaks['source']} burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
+                           + (" x 2, the nominal e4m3/bf16 ratio" if fp8 else "")
+                           + f"; frac of sustained {achieved / (peak * peaks['bf16_tflops_sustained'] / peaks['bf16_tflops']):.3f}"),
+            "algorithmic_bytes_per_launch": alg_bytes}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
             "config": _config(w, res["sets"], res["resident_mb"]),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peaks["bf16_tflops"],
             "roofline": roof, "clocks": sampler.summary(), "gpu_launches": res["launches"]}
@@ -523,7 +565,7 @@ def run_ours(args):
                          "peak_gbs": peaks["hbm_gbs"]}
 
     if rank == 0 or ws > 1:
-        line["e2e"] = e2e_throughput(pa, w, steps=max(3, min(args.steps, 20)), device=device)
+        line["e2e"] = e2e_throughput(pa, w, steps=max(3, min(args.steps, 20)), device=device, fp8=fp8)
         if ws > 1:
             line["e2e"]["value"] = max_over_ranks(-line["e2e"]["value"], device) * -1 * ws
 
@@ -670,6 +712,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="flux", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the e4m3 forward (pa_attn_fwd_fp8) instead of bf16; one-chunk workloads")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (same sequence shape, smaller case; for profiling)")
     ap.add_argument("--no-extra", action="store_true")
