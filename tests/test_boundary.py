@@ -212,3 +212,23 @@ def test_quantize_and_fp8_dev_argument_checks(lib):
     assert call(sk=0) == B.PA_ERR_INVALID_ARG
     assert call(sv=A + 5 * MB + 9) == B.PA_ERR_MISALIGNED
     assert call(d=64) == B.PA_ERR_UNSUPPORTED
+
+
+def test_plain_c_caller(lib, tmp_path):
+    """A C program compiled with gcc against the header and linked to the
+    library gets the documented status codes (no Python in between)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = os.path.join(ROOT, "tests", "c", "abi_smoke.c")
+    exe = str(tmp_path / "abi_smoke")
+    libdir = os.path.dirname(B.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-O1", f"-I{os.path.join(ROOT, 'include')}", src,
+                        "-o", exe, f"-L{libdir}", "-l:libpa_attn.so", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "C ABI checks passed" in r.stdout
