@@ -556,7 +556,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
             "config": _config(w, res["sets"], res["resident_mb"]),
-            "pct_of_bf16_peak": 100.0 * (value / ws) / peaks["bf16_tflops"],
+            ("pct_of_e4m3_peak" if fp8 else "pct_of_bf16_peak"): 100.0 * (value / ws) / peak,
             "roofline": roof, "clocks": sampler.summary(), "gpu_launches": res["launches"]}
     if res["merge_ms"]:
         mb = workloads.merge_bytes(len(w.chunks), w.B, w.H, w.Nq, w.d)
