@@ -82,6 +82,8 @@ def test_workload_table_matches_spec():
     assert (t.B, t.Nq, sum(t.chunks), t.chunks) == (2, 4603, 4603, (1151, 1151, 1151, 1150))
     h = workloads.get("hunyuan")
     assert h.Nq == 33 * 45 * 80 + 256 and sum(workloads.HUNYUAN_CHUNKS8) == h.Nk
+    h8 = workloads.get("hunyuan8")
+    assert h8.chunks == workloads.HUNYUAN_CHUNKS8 and (h8.Nq, h8.seed) == (h.Nq, h.seed)
     a = workloads.get("flux1008")
     assert a.Nq == 63 * 63 + 512 and a.chunks == (1121, 1121, 1121, 1118)
     for w in workloads.WORKLOADS.values():

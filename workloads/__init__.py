@@ -79,6 +79,8 @@ WORKLOADS: Dict[str, Workload] = {
 
 # The 8-chunk split of the HunyuanVideo-shaped workload (ring_degree = 8).
 HUNYUAN_CHUNKS8 = (14882,) * 8
+WORKLOADS["hunyuan8"] = dataclasses.replace(WORKLOADS["hunyuan"], name="hunyuan8", chunks=HUNYUAN_CHUNKS8,
+                                            note="HunyuanVideo shape split over 8 ranks: 8 chunks of 14882")
 
 
 def get(name: str) -> Workload:
