@@ -48,7 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     "source_sha256": "c04f091c8d0496fe9c6bf43b9be3785dd74a359bc103c5c2b6d94497361b1e65",
     "bytes_per_launch": 84987392 + 5752576,   # dram__bytes_read.sum + dram__bytes_write.sum
-    "capture": "profiles/attn_fwd_flux.md",
+    "capture": "ncu --set full, FLUX shape, bench.py --steps 20 --warmup 5 --no-extra --no-cpu-baseline",
 }
 
 
