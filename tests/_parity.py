@@ -1,8 +1,9 @@
 """Comparison helpers shared by the GPU parity tests.
 
 Tolerances (the acceptance bar for floating point in this project): on O,
-max |o_gpu - o_ref| <= 1e-2 and mean |o_gpu - o_ref| <= 1e-3; on LSE, |lse_gpu - lse_ref| / max(|lse_ref|, 1) <= 1e-3 for
-every row.  As a stricter diagnostic, the relative L2 error of O is also held
+max |o_gpu - o_ref| <= 1e-2 and mean |o_gpu - o_ref| <= 1e-3; on LSE,
+|lse_gpu - lse_ref| / max(|lse_ref|, 1) <= 1e-3 for every row.  As a
+stricter diagnostic, the relative L2 error of O is also held
 to <= 1e-2 (derivation: P is rounded to bf16 before P.V, a relative error of
 at most 2^-9 per weight that averages out over keys, and O is rounded to bf16
 on output, 2^-9 relative; together well under 1e-2).
