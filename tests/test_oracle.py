@@ -469,3 +469,16 @@ def test_e4m3_quantize_matches_torch_cast():
     assert np.array_equal(codes[ok], tc)
     assert scale == np.float32(np.max(np.abs(x)) / np.float32(448.0))
     assert E.quantize(np.zeros(7))[1] == 1.0 and not np.any(E.quantize(np.zeros(7))[0])
+
+
+def test_uneven_ring_split_equals_unchunked():
+    # the uneven-tails split of the context-parallel guide's ring-anything
+    # case (4603 keys over 4 ranks), at a small width: chunk + merge = whole
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((1, 2, 48, 8))
+    k = rng.standard_normal((1, 2, 4603, 8))
+    v = rng.standard_normal((1, 2, 4603, 8))
+    o_full, l_full = oracle.attention(q, k, v, 0.35)
+    o_cm, l_cm, parts = oracle.chunked_attention(q, k, v, 0.35, [1151, 1151, 1151, 1150])
+    assert len(parts) == 4
+    assert np.allclose(o_cm, o_full, rtol=0, atol=1e-12) and np.allclose(l_cm, l_full, rtol=0, atol=1e-12)
