@@ -24,12 +24,15 @@ PA_ERR_UNSUPPORTED = -2
 PA_ERR_MISALIGNED = -3
 PA_ERR_CUDA = -4
 PA_ERR_TIMEOUT = -5
+PA_ERR_BAD_INPUT = -6
+PA_ACCUM_FIRST = 1
+PA_ACCUM_FINAL = 2
 
 # (name, restype, argtypes) for every symbol declared in include/pa_attn.h.
 _VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "pa_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
-    "pa_attn_fwd_pair": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
+    "pa_attn_fwd_accum": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP]),
     "pa_attn_fwd_fp8": (_I, [_VP, _VP, _VP, _F, _F, _F, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_fwd_fp8_dev": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP]),
     "pa_quantize_e4m3": (_I, [_VP, ctypes.c_longlong, _VP, _VP, _VP]),
@@ -40,6 +43,7 @@ SIGNATURES = {
     "pa_last_error": (ctypes.c_char_p, []),
     "pa_poll_device_status": (_I, []),
     "pa_selftest_timeout": (_I, [_I, _VP]),
+    "pa_set_wait_limit_ms": (_I, [_I]),
     "pa_version": (_I, []),
 }
 
@@ -88,9 +92,19 @@ def version() -> int:
     return int(load_library().pa_version())
 
 
-def _check(rc: int, where: str) -> None:
+def _check(rc: int, where: str, check: bool = False) -> None:
+    """Raise on a non-zero status.  With ``check`` also wait for the device
+    and raise on an error the kernels recorded (a bounded wait that gave up,
+    a bad value read on the device): this synchronises, so it is for
+    debugging and tests, not for a hot loop."""
     if rc != PA_OK:
         raise PaError(rc, where, last_error())
+    if check:
+        import torch
+        torch.cuda.synchronize()
+        code = poll_device_status()
+        if code != PA_OK:
+            raise PaError(code, where, "reported by the device after the call")
 
 
 def _stream_handle(stream, device) -> int:
@@ -114,12 +128,12 @@ def _check_bf16(name, t, ndim):
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
 
 
-def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=None, pair: bool = False):
+def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=None, check: bool = False):
     """Attention of q [B,H,Nq,d] against one K/V chunk k, v [B,H,Nk,d].
 
     Returns (o [B,H,Nq,d] bf16, lse [B,H,Nq] fp32, natural log), written into
-    ``out`` / ``lse`` when given.  ``scale`` defaults to 1/sqrt(d).  With
-    ``pair=True`` the CTA-pair kernel (``pa_attn_fwd_pair``, d = 128) runs.
+    ``out`` / ``lse`` when given.  ``scale`` defaults to 1/sqrt(d).
+    ``check=True`` synchronises and raises on a device-side error.
     """
     _check_bf16("q", q, 4)
     _check_bf16("k", k, 4)
@@ -131,16 +145,52 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out, lse = _outputs(q, out, lse)
-    lib = load_library()
-    fn = lib.pa_attn_fwd_pair if pair else lib.pa_attn_fwd
-    rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
-            float(scale), _stream_handle(stream, q.device))
-    _check(rc, "pa_attn_fwd_pair" if pair else "pa_attn_fwd")
+    rc = load_library().pa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                     B, H, Nq, Nk, d, float(scale), _stream_handle(stream, q.device))
+    _check(rc, "pa_attn_fwd", check)
     return out, lse
 
 
+def attn_fwd_accum(q, k, v, o_acc, lse_acc, first: bool = False, final: bool = False, out=None,
+                   scale: Optional[float] = None, stream=None, check: bool = False):
+    """Fold the attention of q over one more K/V chunk into the running state
+    (``pa_attn_fwd_accum``): o_acc [B,H,Nq,d] fp32 and lse_acc [B,H,Nq] fp32,
+    updated in place.  ``first`` ignores their incoming contents.  With
+    ``final`` the result goes to ``out`` (bf16, allocated when None) instead
+    of o_acc, and that tensor is returned; otherwise o_acc is returned.
+    Returns (o, lse_acc)."""
+    import torch
+    _check_bf16("q", q, 4)
+    _check_bf16("k", k, 4)
+    _check_bf16("v", v, 4)
+    B, H, Nq, d = q.shape
+    if k.shape[:2] != (B, H) or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    for name, t, shape in (("o_acc", o_acc, (B, H, Nq, d)), ("lse_acc", lse_acc, (B, H, Nq))):
+        if (not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or tuple(t.shape) != shape
+                or not t.is_contiguous() or t.device != q.device):
+            raise ValueError(f"{name} must be a contiguous float32 tensor of shape {shape} on q's device")
+    if final:
+        if out is None:
+            out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+        else:
+            _check_bf16("out", out, 4)
+            if tuple(out.shape) != (B, H, Nq, d):
+                raise ValueError("out must have q's shape")
+    elif out is not None:
+        raise ValueError("out is written only by the final fold")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    flags = (PA_ACCUM_FIRST if first else 0) | (PA_ACCUM_FINAL if final else 0)
+    rc = load_library().pa_attn_fwd_accum(q.data_ptr(), k.data_ptr(), v.data_ptr(), o_acc.data_ptr(),
+                                           lse_acc.data_ptr(), out.data_ptr() if final else None, B, H, Nq,
+                                           k.shape[2], d, float(scale), flags, _stream_handle(stream, q.device))
+    _check(rc, "pa_attn_fwd_accum", check)
+    return (out if final else o_acc), lse_acc
+
+
 def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, scale: Optional[float] = None,
-                 out=None, lse=None, stream=None):
+                 out=None, lse=None, stream=None, check: bool = False):
     """Attention over e4m3 inputs (``pa_attn_fwd_fp8``): q [B,H,Nq,128],
     k, v [B,H,Nk,128] of dtype torch.float8_e4m3fn, whose real values are the
     tensors times their scales.  Returns (o bf16, lse fp32) like attn_fwd."""
@@ -165,16 +215,16 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, scale:
         rc = load_library().pa_attn_fwd_fp8_dev(q.data_ptr(), k.data_ptr(), v.data_ptr(), *[x.data_ptr() for x in scales],
                                                 out.data_ptr(), lse.data_ptr(), B, H, Nq, k.shape[2], d, float(scale),
                                                 _stream_handle(stream, q.device))
-        _check(rc, "pa_attn_fwd_fp8_dev")
+        _check(rc, "pa_attn_fwd_fp8_dev", check)
         return out, lse
     rc = load_library().pa_attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
                                         float(v_scale), out.data_ptr(), lse.data_ptr(), B, H, Nq, k.shape[2], d,
                                         float(scale), _stream_handle(stream, q.device))
-    _check(rc, "pa_attn_fwd_fp8")
+    _check(rc, "pa_attn_fwd_fp8", check)
     return out, lse
 
 
-def quantize_e4m3(x, out=None, scale=None, stream=None):
+def quantize_e4m3(x, out=None, scale=None, stream=None, check: bool = False):
     """Per-tensor e4m3 quantisation of a bf16 tensor on the device
     (``pa_quantize_e4m3``): returns (q torch.float8_e4m3fn of x's shape,
     scale one-element float32 device tensor) with x ~= scale * q."""
@@ -192,11 +242,11 @@ def quantize_e4m3(x, out=None, scale=None, stream=None):
         raise ValueError("scale must be a one-element float32 tensor")
     rc = load_library().pa_quantize_e4m3(x.data_ptr(), x.numel(), out.data_ptr(), scale.data_ptr(),
                                          _stream_handle(stream, x.device))
-    _check(rc, "pa_quantize_e4m3")
+    _check(rc, "pa_quantize_e4m3", check)
     return out, scale
 
 
-def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
+def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None, check: bool = False):
     """Merge n partial results o_parts [n,B,H,N,d] bf16, lse_parts [n,B,H,N]
     fp32 (over disjoint key chunks) into (o [B,H,N,d], lse [B,H,N])."""
     import torch
@@ -218,7 +268,7 @@ def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
     rc = load_library().pa_attn_merge(o_parts.data_ptr(), lse_parts.data_ptr(), n, out.data_ptr(),
                                       lse.data_ptr(), B, H, N, d,
                                       _stream_handle(stream, o_parts.device))
-    _check(rc, "pa_attn_merge")
+    _check(rc, "pa_attn_merge", check)
     return out, lse
 
 
@@ -256,7 +306,8 @@ def _chunk_arrays(q, k_chunks, v_chunks):
     return kp, vp, nk, n
 
 
-def attn_fwd_chunks(q, k_chunks, v_chunks, scale: Optional[float] = None, out=None, lse=None, stream=None):
+def attn_fwd_chunks(q, k_chunks, v_chunks, scale: Optional[float] = None, out=None, lse=None, stream=None,
+                    check: bool = False):
     """Attention of q over the concatenation of the K/V chunks (up to 8) in a
     single launch (``pa_attn_fwd_chunks``); no partial results are written."""
     _check_bf16("q", q, 4)
@@ -267,11 +318,12 @@ def attn_fwd_chunks(q, k_chunks, v_chunks, scale: Optional[float] = None, out=No
     out, lse = _outputs(q, out, lse)
     rc = load_library().pa_attn_fwd_chunks(q.data_ptr(), kp, vp, nk, n, out.data_ptr(), lse.data_ptr(),
                                            B, H, Nq, d, float(scale), _stream_handle(stream, q.device))
-    _check(rc, "pa_attn_fwd_chunks")
+    _check(rc, "pa_attn_fwd_chunks", check)
     return out, lse
 
 
-def attn_chunks_noalloc(q, k_chunks, v_chunks, scale: Optional[float] = None, out=None, lse=None, stream=None):
+def attn_chunks_noalloc(q, k_chunks, v_chunks, scale: Optional[float] = None, out=None, lse=None, stream=None,
+                        check: bool = False):
     """Attention of q over the concatenation of the K/V chunks through
     ``pa_attn_chunks_noalloc``: the library keeps the per-chunk partials in
     its fixed static array instead of allocating them (see the header for the
@@ -285,7 +337,7 @@ def attn_chunks_noalloc(q, k_chunks, v_chunks, scale: Optional[float] = None, ou
     out, lse = _outputs(q, out, lse)
     rc = load_library().pa_attn_chunks_noalloc(q.data_ptr(), kp, vp, nk, n, out.data_ptr(), lse.data_ptr(),
                                                B, H, Nq, d, float(scale), _stream_handle(stream, q.device))
-    _check(rc, "pa_attn_chunks_noalloc")
+    _check(rc, "pa_attn_chunks_noalloc", check)
     return out, lse
 
 
@@ -293,6 +345,12 @@ def poll_device_status() -> int:
     """Read and clear the device status word (synchronising).  Returns the
     status code (0 = no device-side error since the last poll)."""
     return int(load_library().pa_poll_device_status())
+
+
+def set_wait_limit_ms(ms: int) -> None:
+    """Limit of every device-side barrier wait for later launches
+    (``pa_set_wait_limit_ms``; default 5000 ms)."""
+    _check(load_library().pa_set_wait_limit_ms(int(ms)), "pa_set_wait_limit_ms")
 
 
 def selftest_timeout(limit_us: int, stream=None) -> None:

@@ -22,7 +22,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libpa_attn.so")
 SOURCES = [os.path.join(CSRC, "pa_attn.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "fwd_common.cuh", "attn_fwd.cuh", "attn_fwd_pair.cuh", "lse_merge.cuh", "quantize.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "fwd_common.cuh", "attn_fwd.cuh", "lse_merge.cuh", "quantize.cuh")] + [
     os.path.join(INCLUDE, "pa_attn.h")]
 
 NVCC_FLAGS = [

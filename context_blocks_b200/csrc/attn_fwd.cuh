@@ -25,8 +25,15 @@
 //   [256+D,256+2D) O_1 accumulator
 // Thread t of softmax warpgroup i owns TMEM lane t = query row t of tile i,
 // so row max, row sum and rescaling need no cross-thread reduction.  Each
-// warpgroup hands P to the MMA warp in two halves (PA_SPLIT_P), so P.V on the
-// first 64 keys starts while the second half is still being computed.
+// warpgroup hands P to the MMA warp in two halves, so P.V on the first 64
+// keys starts while the second half is still being computed.
+//
+// Accumulate mode (FwdParams::acc_o set): the launch folds its chunk into a
+// caller-owned running state, a normalised fp32 O and its LSE.  That state is
+// exactly (O_unnormalised = O, l = 1, m = LSE * log2(e)) in the online softmax
+// below, so the softmax threads load it into the O accumulator before the
+// first tile and carry on; the epilogue writes the updated state back (or,
+// on the final fold, the bf16 output).
 //
 // With kFp8 the same kernel takes e4m3 Q, K, V (per-tensor scales folded into
 // the logit scale and the epilogue) and issues kind::f8f6f4 MMAs.
@@ -46,40 +53,12 @@
 namespace pa {
 namespace single {
 
-// Softmax arithmetic variants, measured against each other (all compute the
-// same values up to rounding order):
-//   PA_SINGLE_MAX3    row max as 8 chains of 3-input max instead of one chain
-//   PA_SINGLE_F2      scale-and-subtract and row sum on packed f32x2 pairs,
-//                     row sum in 4 partial sums
-//   PA_SINGLE_EMU     one exponential pair in PA_SINGLE_EMU on the FMA pipe
-//                     (exp2_poly_x2), 0 = all on MUFU
-#ifndef PA_SINGLE_MAX3
-#define PA_SINGLE_MAX3 1
-#endif
-#ifndef PA_SINGLE_F2
-#define PA_SINGLE_F2 1
-#endif
-#ifndef PA_SINGLE_EMU
-#define PA_SINGLE_EMU 0
-#endif
-//   PA_SPLIT_P        P handed to the MMA warp in this many parts (1, 2 or 4)
-//                     of the key tile, so P.V on the first parts runs while
-//                     the later ones are computed
-#ifndef PA_SPLIT_P
-#define PA_SPLIT_P 2
-#endif
-constexpr int kPParts = PA_SPLIT_P;
-static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P is handed over in 1, 2 or 4 parts");
-// Barrier waits:
-//   PA_WAIT_HINT      waits of the softmax warps and of the MMA-issuing thread
-//                     pass a long suspend-time hint to mbarrier.try_wait, so a
-//                     waiting thread sleeps until the phase completes instead
-//                     of probing the barrier again and again
-#ifndef PA_WAIT_HINT
-#define PA_WAIT_HINT 1
-#endif
+// Waits of the softmax warps and of the MMA-issuing warp pass this
+// suspend-time hint to mbarrier.try_wait: a waiting thread sleeps until the
+// phase completes instead of probing the barrier again and again.
 constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms; the wait itself stays bounded by the time limit
 
+constexpr int kPParts = 2;         // P is handed to the MMA warp in this many parts
 constexpr int kStages = 4;         // K/V ring slots (each holds one K or one V tile)
 constexpr int kMaxChunks = 8;      // K/V chunks one launch can consume
 
@@ -291,11 +270,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     };
     auto wait_all = [&](uint32_t bar, uint32_t parity) {
-      const bool got = PA_WAIT_HINT ? mbar_wait_hint(bar, parity, abort_word, p.status, kStatusTimeout, lim,
-                                                     kSuspendHintNs)
-                                    : mbar_wait(bar, parity, abort_word, p.status, kStatusTimeout, lim);
+      const bool got = mbar_wait_hint(bar, parity, abort_word, p.status, kStatusTimeout, lim, kSuspendHintNs);
       return __all_sync(0xffffffffu, got);
     };
+    // With a running state loaded into O (accumulate mode) even the first
+    // P.V accumulates.
+    const bool o_loaded = (p.acc_o != nullptr) && !(p.acc_flags & kAccFirst);
 
     bool ok = wait_all(bar_q_full0, 0) && wait_all(bar_q_full0 + 8, 0) && wait_all(bar_kv_full0, 0);
     if (ok) {
@@ -335,7 +315,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             break;
           }
           tc_fence_after();
-          if (leader) issue_pv(i, sv, j > 0 || q > 0, q * kKkPerPart, (q + 1) * kKkPerPart);
+          if (leader) issue_pv(i, sv, o_loaded || j > 0 || q > 0, q * kKkPerPart, (q + 1) * kKkPerPart);
           __syncwarp();
         }
         if (!ok || !wait_all(bar_p_full0 + 8 * i, j & 1)) {
@@ -343,7 +323,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           break;
         }
         tc_fence_after();
-        if (leader) issue_pv(i, sv, j > 0 || kPParts > 1, (kPParts - 1) * kKkPerPart, kBN / kKPerMma);
+        if (leader) issue_pv(i, sv, true, (kPParts - 1) * kKkPerPart, kBN / kKPerMma);
         if (leader && i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
         __syncwarp();
         if (more) {
@@ -378,13 +358,56 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tS = tmem + i * kBN + lane_off;
     const uint32_t tO = tmem + 2 * kBN + i * D + lane_off;
     const int row = q0 + i * kBM + t;
+    const bool in_range = row < p.Nq;
+    const size_t row_idx = static_cast<size_t>(bh) * p.Nq + row;
     // Logit scale in log2 units; e4m3 inputs may carry their dequantisation
-    // scales in device memory.
+    // scales in device memory, which are checked here: a scale that is not
+    // finite and positive is reported in the status word (the outputs are then
+    // meaningless, as the header says).
     float c = p.scale_log2;
-    if constexpr (kFp8) c *= (p.dscale_q != nullptr) ? __ldg(p.dscale_q) * __ldg(p.dscale_k) : p.qk_scale;
+    float o_mul = 1.f;
+    if constexpr (kFp8) {
+      if (p.dscale_q != nullptr) {
+        const float sq = __ldg(p.dscale_q), sk = __ldg(p.dscale_k), sv = __ldg(p.dscale_v);
+        const bool good = (sq > 0.f && sq <= FLT_MAX) && (sk > 0.f && sk <= FLT_MAX) && (sv > 0.f && sv <= FLT_MAX);
+        if (!good && threadIdx.x == 0) atomicCAS(p.status, 0, kStatusBadInput);
+        c *= sq * sk;
+        o_mul = sv;
+      } else {
+        c *= p.qk_scale;
+        o_mul = p.o_scale;
+      }
+    }
     float m_ref = -INFINITY;
     float l = 0.f;
     bool ok = true;
+    // Accumulate mode: start from the caller's running (O, LSE) instead of an
+    // empty state.  Rows past Nq and rows whose running LSE is -inf (no key
+    // seen yet) start empty, with O = 0.
+    const bool o_loaded = (p.acc_o != nullptr) && !(p.acc_flags & kAccFirst);
+    if (o_loaded) {
+      const float lse0 = in_range ? p.acc_lse[row_idx] : -INFINITY;
+      const bool have = lse0 > -INFINITY;
+      if (have) {
+        m_ref = lse0 * 1.4426950408889634f;
+        l = 1.f;
+      }
+      const float4* src = reinterpret_cast<const float4*>(p.acc_o + row_idx * D);
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t orr[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 x = have ? __ldg(src + ch * 8 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+          orr[4 * v] = __float_as_uint(x.x);
+          orr[4 * v + 1] = __float_as_uint(x.y);
+          orr[4 * v + 2] = __float_as_uint(x.z);
+          orr[4 * v + 3] = __float_as_uint(x.w);
+        }
+        tmem_st_x32(tO + ch * 32, orr);
+      }
+      tmem_st_wait();
+    }
 
     for (int j = 0; j < n; ++j) {
       // Chunk of key tile j, from the prefix tile counts (no state carried).
@@ -393,9 +416,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int cc = 1; cc < kMaxChunks; ++cc) chunk += (j >= kv.tile_start[cc]) ? 1 : 0;
       const int valid = kv.nk[chunk] - (j - kv.tile_start[chunk]) * kBN;  // keys of this tile in its chunk
       const bool got =
-          PA_WAIT_HINT
-              ? mbar_wait_hint(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim, kSuspendHintNs)
-              : mbar_wait(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim);
+          mbar_wait_hint(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim, kSuspendHintNs);
       if (__any_sync(0xffffffffu, !got)) {
         ok = false;
         break;
@@ -406,13 +427,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float s[kBN];
 #pragma unroll
       for (int e = 0; e < kBN; ++e) s[e] = __uint_as_float(sr[e]);
-      const bool full_tile = valid >= kBN;  // tail tiles keep every exponential on MUFU
       if (valid < kBN) {
 #pragma unroll
         for (int e = 0; e < kBN; ++e)
           if (e >= valid) s[e] = -INFINITY;
       }
-#if PA_SINGLE_MAX3
+      // Row max: 8 independent chains of 3-input max.
       float m8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
@@ -421,23 +441,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) m8[k] = max3f(m8[k], s[e + k], s[e + 8 + k]);
       float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], max3f(m8[5], m8[6], m8[7])));
-#else
-      float mx = s[0];
-#pragma unroll
-      for (int e = 1; e < kBN; ++e) mx = fmaxf(mx, s[e]);
-#endif
       mx *= c;
       float alpha = 1.f;
       bool rescale = false;
       if (mx > m_ref + kRescaleLog2) {
-        alpha = ex2_approx(m_ref - mx);  // 0 on the first tile (m_ref = -inf)
+        alpha = ex2_approx(m_ref - mx);  // 0 when the row was empty (m_ref = -inf)
         l *= alpha;
         m_ref = mx;
-        rescale = (j > 0);
+        rescale = (j > 0) || o_loaded;
       }
       if (__any_sync(0xffffffffu, rescale)) {
         // PV of tile j-1 has completed: S_i(j) was issued after it and the
-        // tcgen05 ops of the issuing thread complete in order.
+        // tcgen05 ops of the issuing thread complete in order.  (On tile 0 of
+        // a fold, O holds the loaded state this thread stored.)
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t orr[32];
@@ -447,39 +463,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tmem_st_x32(tO + ch * 32, orr);
         }
       }
+      // x = s * c - m_ref on packed pairs, P = 2^x on MUFU, the row sum in
+      // four packed partial sums.
       const float neg_m = -m_ref;
-#if PA_SINGLE_F2
       const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
       uint64_t l4[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-#endif
 #pragma unroll
       for (int ch = 0; ch < kBN / 32; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float p0, p1;
-#if PA_SINGLE_F2
-          const uint64_t x = f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2);
-          if (PA_SINGLE_EMU > 0 && full_tile && (e % (PA_SINGLE_EMU > 0 ? PA_SINGLE_EMU : 1)) == 0) {
-            f2_split(exp2_poly_x2(x), p0, p1);
-          } else {
-            float x0, x1;
-            f2_split(x, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
+          float x0, x1;
+          f2_split(f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
           l4[e & 3] = f2_add(l4[e & 3], f2(p0, p1));
-#else
-          const float x0 = fmaf(s[ch * 32 + 2 * e], c, neg_m);
-          const float x1 = fmaf(s[ch * 32 + 2 * e + 1], c, neg_m);
-          if (PA_SINGLE_EMU > 0 && full_tile && (e % (PA_SINGLE_EMU > 0 ? PA_SINGLE_EMU : 1)) == 0) {
-            f2_split(exp2_poly_x2(f2(x0, x1)), p0, p1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          l += p0 + p1;
-#endif
           if constexpr (kFp8) {
             // four e4m3 keys per 32-bit column, lowest key in the low byte
             const uint32_t h = pack_e4m3x2(p0, p1);
@@ -498,7 +496,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tmem_st_x16(tS + ch * 16, pk);
         }
         constexpr int kChPerPart = (kBN / 32) / kPParts;  // 32-key chunks per part
-        if (kPParts > 1 && (ch + 1) % kChPerPart == 0 && ch + 1 < kBN / 32) {
+        if ((ch + 1) % kChPerPart == 0 && ch + 1 < kBN / 32) {
           // Part (ch + 1) / kChPerPart - 1 of P is in TMEM: hand it over.
           tmem_st_wait();
           tc_fence_before();
@@ -506,14 +504,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (lane == 0) mbar_arrive(bar_p_part0 + 8 * (3 * i + (ch + 1) / kChPerPart - 1));
         }
       }
-#if PA_SINGLE_F2
       {
-        const uint64_t t = f2_add(f2_add(l4[0], l4[1]), f2_add(l4[2], l4[3]));
+        const uint64_t sum = f2_add(f2_add(l4[0], l4[1]), f2_add(l4[2], l4[3]));
         float a, b;
-        f2_split(t, a, b);
+        f2_split(sum, a, b);
         l += a + b;
       }
-#endif
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -526,27 +522,48 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      float inv_l = 1.f / l;
-      if constexpr (kFp8) inv_l = ((p.dscale_v != nullptr) ? __ldg(p.dscale_v) : p.o_scale) / l;
-      const bool in_range = row < p.Nq;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.Nq + row) * D;
+      const float inv_l = o_mul / l;
+      const float lse_out = (m_ref + lg2_approx(l)) * 0.69314718055994531f;
+      const bool state_out = (p.acc_o != nullptr) && !(p.acc_flags & kAccFinal);
+      if (state_out) {
+        // Running state: normalised fp32 O and its LSE.
+        float4* dst = reinterpret_cast<float4*>(p.acc_o + row_idx * D);
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t orr[32];
-        tmem_ld_x32(tO + ch * 32, orr);
-        uint32_t pk[16];
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t orr[32];
+          tmem_ld_x32(tO + ch * 32, orr);
+          if (in_range) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
-        if (in_range) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+            for (int v = 0; v < 8; ++v)
+              dst[ch * 8 + v] = make_float4(__uint_as_float(orr[4 * v]) * inv_l, __uint_as_float(orr[4 * v + 1]) * inv_l,
+                                            __uint_as_float(orr[4 * v + 2]) * inv_l,
+                                            __uint_as_float(orr[4 * v + 3]) * inv_l);
+          }
+        }
+      } else {
+        __nv_bfloat16* orow = p.o + row_idx * D;
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t orr[32];
+          tmem_ld_x32(tO + ch * 32, orr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
+          if (in_range) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
       }
-      if (in_range)
-        p.lse[static_cast<size_t>(bh) * p.Nq + row] = (m_ref + lg2_approx(l)) * 0.69314718055994531f;
+      if (in_range) {
+        if (p.acc_o != nullptr)
+          p.acc_lse[row_idx] = lse_out;
+        else
+          p.lse[row_idx] = lse_out;
+      }
     }
   }
 

@@ -1,9 +1,9 @@
-// Definitions shared by the forward kernels (attn_fwd.cuh, attn_fwd_pair.cuh):
-// tile sizes, launch parameters and the small arithmetic helpers of the
-// online softmax.
+// Definitions shared by the forward kernels: tile sizes, launch parameters
+// and the small arithmetic helpers of the online softmax.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cfloat>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -20,6 +20,11 @@ constexpr float kRescaleLog2 = 8.0f;
 
 // Device status codes written by kernels (mirror PA_ERR_* in pa_attn.h).
 constexpr int kStatusTimeout = -5;
+constexpr int kStatusBadInput = -6;
+
+// Accumulate-mode flags (FwdParams::acc_flags; PA_ACCUM_* in pa_attn.h).
+constexpr int kAccFirst = 1;   // no incoming state: start from an empty one
+constexpr int kAccFinal = 2;   // write the bf16 output instead of the fp32 state
 
 struct FwdParams {
   __nv_bfloat16* o;     // [B*H, Nq, D]
@@ -37,6 +42,12 @@ struct FwdParams {
   const float* dscale_q;
   const float* dscale_k;
   const float* dscale_v;
+  // Accumulate mode (acc_o != null): acc_o [B*H, Nq, D] fp32 and acc_lse
+  // [B*H, Nq] hold the running (normalised O, LSE) that the launch folds its
+  // keys into; `lse` is unused and `o` is written only with kAccFinal.
+  float* acc_o;
+  float* acc_lse;
+  int acc_flags;
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -79,38 +90,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^x on the FMA pipe for both halves of a pair, to take load off the MUFU
-// unit.  Range reduction x = n + f with n = round-to-nearest(x) (adding and
-// subtracting 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
-// (coefficients from gen_exp2_poly.py: minimax in relative error, 7.6e-5 on
-// the reduced range); 2^n by adding n to the exponent field.  x is clamped to
-// >= -126 so that the exponent add cannot underflow into the sign bit; the
-// result for smaller x is ~2^-126, i.e. zero at the precision P is kept in.
-constexpr float kExp2C0 = 9.999275804e-01f;
-constexpr float kExp2C1 = 6.932516098e-01f;
-constexpr float kExp2C2 = 2.426152676e-01f;
-constexpr float kExp2C3 = 5.522262305e-02f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  float a, b;
-  f2_split(x, a, b);
-  const uint64_t xc = f2(fmaxf(a, -126.f), fmaxf(b, -126.f));
-  const uint64_t t = f2_add(xc, f2(kRoundMagic, kRoundMagic));        // magic + n
-  const uint64_t n = f2_add(t, f2(-kRoundMagic, -kRoundMagic));       // n (exact)
-  const uint64_t fr = f2_fma(n, f2(-1.f, -1.f), xc);                  // f = x - n (exact)
-  uint64_t p = f2_fma(f2(kExp2C3, kExp2C3), fr, f2(kExp2C2, kExp2C2));
-  p = f2_fma(p, fr, f2(kExp2C1, kExp2C1));
-  p = f2_fma(p, fr, f2(kExp2C0, kExp2C0));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  // low bits of t hold n; shifting by 23 moves n into the exponent field
-  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-  return f2(r0, r1);
 }
 
 }  // namespace pa

@@ -8,10 +8,11 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "attn_fwd.cuh"
-#include "attn_fwd_pair.cuh"
 #include "quantize.cuh"
 #include "fwd_common.cuh"
 #include "lse_merge.cuh"
@@ -46,8 +47,11 @@ __global__ void timeout_probe_kernel(unsigned long long limit_ns, int* status) {
 
 namespace {
 
-constexpr unsigned long long kDefaultTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s
+constexpr int kDefaultWaitLimitMs = 5000;
 constexpr int kMaxDevices = 64;
+
+// Limit of every device-side barrier wait, in nanoseconds (pa_set_wait_limit_ms).
+std::atomic<unsigned long long> g_wait_limit_ns{static_cast<unsigned long long>(kDefaultWaitLimitMs) * 1000000ull};
 
 thread_local char g_err[512] = "";
 
@@ -70,7 +74,6 @@ struct DeviceState {
   int* status = nullptr;  // device address of pa::g_status
   unsigned char* noalloc_scratch = nullptr;  // device address of pa::g_noalloc_scratch
   bool fwd_attr[3] = {false, false, false};  // d = 64, d = 128, e4m3 d = 128
-  bool pair_attr = false;
 };
 
 
@@ -168,13 +171,22 @@ int encode_map(CUtensorMap* map, const void* ptr, int d, int n_rows, int bh, int
   return PA_OK;
 }
 
+// Running state of an accumulating launch (pa_attn_fwd_accum); acc_o null
+// for an ordinary launch.
+struct AccArgs {
+  float* acc_o = nullptr;
+  float* acc_lse = nullptr;
+  int flags = 0;
+};
+
 // Single-CTA forward over n_chunks K/V chunks (n_chunks = 1 for one chunk).
 // kFp8: e4m3 Q/K/V with dequantisation scales; qk_scale multiplies the logits
 // (on top of `scale`) and o_scale the output.
 template <int D, bool kFp8 = false>
 int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void* const* v, const int* nk,
                int n_chunks, void* o, float* lse, int BH, int Nq, float scale, cudaStream_t stream,
-               float qk_scale = 1.f, float o_scale = 1.f, const float* const* dscales = nullptr) {
+               float qk_scale = 1.f, float o_scale = 1.f, const float* const* dscales = nullptr,
+               const AccArgs& acc = AccArgs()) {
   using L = pa::single::FwdLayout<D, kFp8>;
   CUtensorMap tq;
   pa::single::KvChunks kv;
@@ -215,12 +227,15 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   prm.n_kv_tiles = static_cast<int>(tiles_total);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.status = st->status;
-  prm.timeout_ns = kDefaultTimeoutNs;
+  prm.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   prm.qk_scale = qk_scale;
   prm.o_scale = o_scale;
   prm.dscale_q = dscales ? dscales[0] : nullptr;
   prm.dscale_k = dscales ? dscales[1] : nullptr;
   prm.dscale_v = dscales ? dscales[2] : nullptr;
+  prm.acc_o = acc.acc_o;
+  prm.acc_lse = acc.acc_lse;
+  prm.acc_flags = acc.flags;
   dim3 grid((Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM), BH);
   kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, kv, prm);
   cudaError_t e = cudaGetLastError();
@@ -228,62 +243,12 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   return PA_OK;
 }
 
-// CTA-pair forward (head dim 128): clusters of two CTAs, 512 query rows each.
-int launch_fwd_pair(DeviceState* st, const void* q, const void* k, const void* v, void* o, float* lse, int BH,
-                    int Nq, int Nk, float scale, cudaStream_t stream) {
-  using L = pa::pairk::PairLayout;
-  CUtensorMap tq, tk, tv;
-  int rc;
-  if ((rc = encode_map(&tq, q, 128, Nq, BH, pa::kBM)) != PA_OK) return rc;
-  if ((rc = encode_map(&tk, k, 128, Nk, BH, pa::kBN / 2)) != PA_OK) return rc;
-  if ((rc = encode_map(&tv, v, 128, Nk, BH, pa::kBN)) != PA_OK) return rc;
-  auto kern = pa::pairk::attn_fwd_pair_kernel<128>;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!st->pair_attr) {
-      // The kernel re-allocates registers between warpgroups with setmaxnreg;
-      // the split is only valid for the per-thread count it was designed for.
-      cudaFuncAttributes fa;
-      cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-      if (fa.numRegs != pa::pairk::kLaunchRegs)
-        return fail(PA_ERR_UNSUPPORTED, "attn_fwd_pair built with %d registers per thread, expected %d",
-                    fa.numRegs, pa::pairk::kLaunchRegs);
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-      st->pair_attr = true;
-    }
-  }
-  pa::FwdParams prm;
-  prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.lse = lse;
-  prm.Nq = Nq;
-  prm.Nk = Nk;
-  prm.n_kv_tiles = (Nk + pa::kBN - 1) / pa::kBN;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.status = st->status;
-  prm.timeout_ns = kDefaultTimeoutNs;
-  prm.qk_scale = 1.f;
-  prm.o_scale = 1.f;
-  prm.dscale_q = prm.dscale_k = prm.dscale_v = nullptr;
-  const int rows_per_pair = 2 * pa::kQTiles * pa::kBM;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * ((Nq + rows_per_pair - 1) / rows_per_pair), BH);
-  cfg.blockDim = dim3(pa::pairk::kFwdThreads);
-  cfg.dynamicSmemBytes = L::kAllocBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, prm);
-  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_pair launch");
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_pair launch");
-  return PA_OK;
+// The bf16 forward for head dim d (64 or 128).
+int launch_bf16(DeviceState* st, int d, const void* q, const void* const* k, const void* const* v, const int* nk,
+                int n_chunks, void* o, float* lse, int BH, int Nq, float scale, cudaStream_t stream,
+                const AccArgs& acc = AccArgs()) {
+  if (d == 64) return launch_fwd<64>(st, q, k, v, nk, n_chunks, o, lse, BH, Nq, scale, stream, 1.f, 1.f, nullptr, acc);
+  return launch_fwd<128>(st, q, k, v, nk, n_chunks, o, lse, BH, Nq, scale, stream, 1.f, 1.f, nullptr, acc);
 }
 
 template <int D>
@@ -305,11 +270,14 @@ int launch_merge(DeviceState* st, const void* o_parts, const float* lse_parts, i
 
 namespace {
 
-// Argument checks shared by the forward entry points.  On PA_OK, *st is the
-// current device's state, or null when there is nothing to do (Nq == 0).
-int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
-                   int d, float scale, DeviceState** st, bool host_only = false, int in_elem_bytes = 2) {
-  *st = nullptr;
+// Host-side checks of one forward call (no CUDA API touched): pointers, sizes,
+// alignment, and that no output overlaps an input or another output.
+// o_elem_bytes is 2 for a bf16 output, 4 for the fp32 running state of an
+// accumulating call; o2 is a second output of o's shape (the bf16 output of a
+// final fold), or null.
+int host_fwd_checks(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int H,
+                    int Nq, int Nk, int d, float scale, int in_elem_bytes = 2, int o_elem_bytes = 2,
+                    const void* o2 = nullptr) {
   if (!q || !k || !v || !o || !lse) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
   if (B < 1 || H < 1) return fail(PA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
   if (Nq < 0) return fail(PA_ERR_INVALID_ARG, "Nq must be >= 0 (got %d)", Nq);
@@ -318,29 +286,79 @@ int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* 
   if (d != 64 && d != 128) return fail(PA_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 65535) return fail(PA_ERR_UNSUPPORTED, "B*H must be <= 65535 (got %lld)", bh);
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (o2 && !aligned(o2, 16)))
     return fail(PA_ERR_MISALIGNED, "q, k, v and o must be 16-byte aligned");
   if (!aligned(lse, 4)) return fail(PA_ERR_MISALIGNED, "lse must be 4-byte aligned");
   if (Nq == 0) return PA_OK;
   const uint64_t qbytes = static_cast<uint64_t>(bh) * Nq * d * in_elem_bytes;
   const uint64_t kbytes = static_cast<uint64_t>(bh) * Nk * d * in_elem_bytes;
-  const uint64_t obytes = static_cast<uint64_t>(bh) * Nq * d * 2;
+  const uint64_t obytes = static_cast<uint64_t>(bh) * Nq * d * o_elem_bytes;
+  const uint64_t o2bytes = static_cast<uint64_t>(bh) * Nq * d * 2;
   const uint64_t lbytes = static_cast<uint64_t>(bh) * Nq * 4;
   const void* ins[3] = {q, k, v};
   const uint64_t in_bytes[3] = {qbytes, kbytes, kbytes};
   for (int i = 0; i < 3; ++i)
-    if (overlap(ins[i], in_bytes[i], o, obytes) || overlap(ins[i], in_bytes[i], lse, lbytes))
+    if (overlap(ins[i], in_bytes[i], o, obytes) || overlap(ins[i], in_bytes[i], lse, lbytes) ||
+        (o2 && overlap(ins[i], in_bytes[i], o2, o2bytes)))
       return fail(PA_ERR_INVALID_ARG, "outputs overlap an input");
   if (overlap(o, obytes, lse, lbytes)) return fail(PA_ERR_INVALID_ARG, "o and lse overlap");
-  if (host_only) return PA_OK;
+  if (o2 && (overlap(o2, o2bytes, o, obytes) || overlap(o2, o2bytes, lse, lbytes)))
+    return fail(PA_ERR_INVALID_ARG, "o overlaps the running state");
+  return PA_OK;
+}
 
+// Every pointer must be device memory of the current device; on PA_OK *st is
+// that device's state.  Each distinct pointer is queried once.
+int device_checks(const void* const* ptrs, const char* const* names, int n, DeviceState** st) {
   (void)cudaGetLastError();
   int dev = 0, rc;
+  for (int i = 0; i < n; ++i) {
+    bool seen = false;
+    for (int j = 0; j < i && !seen; ++j) seen = (ptrs[j] == ptrs[i]);
+    if (!seen && (rc = check_device_ptr(ptrs[i], names[i], &dev)) != PA_OK) return rc;
+  }
+  return device_state(dev, st);
+}
+
+// Host and device checks of a one-chunk forward.  On PA_OK, *st is the current
+// device's state, or null when there is nothing to do (Nq == 0).
+int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                   int d, float scale, DeviceState** st, int in_elem_bytes = 2) {
+  *st = nullptr;
+  int rc = host_fwd_checks(q, k, v, o, lse, B, H, Nq, Nk, d, scale, in_elem_bytes);
+  if (rc != PA_OK || Nq == 0) return rc;
   const void* ptrs[5] = {q, k, v, o, lse};
   const char* names[5] = {"q", "k", "v", "o", "lse"};
-  for (int i = 0; i < 5; ++i)
-    if ((rc = check_device_ptr(ptrs[i], names[i], &dev)) != PA_OK) return rc;
-  return device_state(dev, st);
+  return device_checks(ptrs, names, 5, st);
+}
+
+// The same for a table of chunks: every chunk's host checks first, so no CUDA
+// call is made for a bad table, then each distinct pointer once.
+int check_chunk_args(const void* q, const void* const* k_chunks, const void* const* v_chunks, const int* nk_chunks,
+                     int n_chunks, int max_chunks, void* o, float* lse, int B, int H, int Nq, int d, float scale,
+                     DeviceState** st) {
+  *st = nullptr;
+  if (!q || !k_chunks || !v_chunks || !nk_chunks || !o || !lse)
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (n_chunks < 1 || n_chunks > max_chunks)
+    return fail(PA_ERR_INVALID_ARG, "n_chunks must be in [1, %d] (got %d)", max_chunks, n_chunks);
+  for (int c = 0; c < n_chunks; ++c) {
+    const int rc = host_fwd_checks(q, k_chunks[c], v_chunks[c], o, lse, B, H, Nq, nk_chunks[c], d, scale);
+    if (rc != PA_OK) return rc;
+  }
+  if (Nq == 0) return PA_OK;
+  constexpr int kMax = 3 + 2 * 64;
+  const void* ptrs[kMax];
+  const char* names[kMax];
+  int n = 0;
+  ptrs[n] = q, names[n++] = "q";
+  ptrs[n] = o, names[n++] = "o";
+  ptrs[n] = lse, names[n++] = "lse";
+  for (int c = 0; c < n_chunks && n + 2 <= kMax; ++c) {
+    ptrs[n] = k_chunks[c], names[n++] = "k chunk";
+    ptrs[n] = v_chunks[c], names[n++] = "v chunk";
+  }
+  return device_checks(ptrs, names, n, st);
 }
 
 }  // namespace
@@ -353,9 +371,27 @@ int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse
   DeviceState* st = nullptr;
   int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st);
   if (rc != PA_OK || st == nullptr) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_fwd<64>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, s);
-  return launch_fwd<128>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, s);
+  return launch_bf16(st, d, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, static_cast<cudaStream_t>(stream));
+}
+
+int pa_attn_fwd_accum(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, void* o, int B,
+                      int H, int Nq, int Nk, int d, float scale, int flags, void* stream) {
+  g_err[0] = '\0';
+  if (flags & ~(PA_ACCUM_FIRST | PA_ACCUM_FINAL)) return fail(PA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const bool final_fold = (flags & PA_ACCUM_FINAL) != 0;
+  if (final_fold && !o) return fail(PA_ERR_INVALID_ARG, "PA_ACCUM_FINAL needs the bf16 output o");
+  if (!final_fold && o) return fail(PA_ERR_INVALID_ARG, "o is written only with PA_ACCUM_FINAL: pass null");
+  int rc = host_fwd_checks(q, k, v, o_acc, lse_acc, B, H, Nq, Nk, d, scale, 2, 4, o);
+  if (rc != PA_OK || Nq == 0) return rc;
+  const void* ptrs[6] = {q, k, v, o_acc, lse_acc, o ? o : o_acc};
+  const char* names[6] = {"q", "k", "v", "o_acc", "lse_acc", "o"};
+  DeviceState* st = nullptr;
+  if ((rc = device_checks(ptrs, names, 6, &st)) != PA_OK) return rc;
+  AccArgs acc;
+  acc.acc_o = o_acc;
+  acc.acc_lse = lse_acc;
+  acc.flags = (flags & PA_ACCUM_FIRST ? pa::kAccFirst : 0) | (final_fold ? pa::kAccFinal : 0);
+  return launch_bf16(st, d, q, &k, &v, &Nk, 1, o, nullptr, B * H, Nq, scale, static_cast<cudaStream_t>(stream), acc);
 }
 
 int pa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale, float v_scale,
@@ -364,10 +400,10 @@ int pa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, 
   for (float sc : {q_scale, k_scale, v_scale})
     if (!std::isfinite(sc) || !(sc > 0.f)) return fail(PA_ERR_INVALID_ARG, "dequantisation scales must be finite and > 0");
   DeviceState* st = nullptr;
-  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, true, 1);  // host-side checks
+  int rc = host_fwd_checks(q, k, v, o, lse, B, H, Nq, Nk, d, scale, 1);
   if (rc != PA_OK) return rc;
   if (d != 128) return fail(PA_ERR_UNSUPPORTED, "the e4m3 forward needs d = 128 (got %d)", d);
-  rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, false, 1);
+  rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, 1);
   if (rc != PA_OK || st == nullptr) return rc;
   return launch_fwd<128, true>(st, q, &k, &v, &Nk, 1, o, lse, B * H, Nq, scale, static_cast<cudaStream_t>(stream),
                                q_scale * k_scale, v_scale);
@@ -381,10 +417,10 @@ int pa_attn_fwd_fp8_dev(const void* q, const void* k, const void* v, const float
   if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
     return fail(PA_ERR_MISALIGNED, "scale pointers must be 4-byte aligned");
   DeviceState* st = nullptr;
-  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, true, 1);  // host-side checks
+  int rc = host_fwd_checks(q, k, v, o, lse, B, H, Nq, Nk, d, scale, 1);
   if (rc != PA_OK) return rc;
   if (d != 128) return fail(PA_ERR_UNSUPPORTED, "the e4m3 forward needs d = 128 (got %d)", d);
-  rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, false, 1);
+  rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st, 1);
   if (rc != PA_OK || st == nullptr) return rc;
   int dev = 0;
   const float* sp[3] = {q_scale, k_scale, v_scale};
@@ -421,7 +457,7 @@ int pa_quantize_e4m3(const void* x, long long n, void* q, float* scale, void* st
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   pa::quant::amax_kernel<<<grid, pa::quant::kThreads, 0, s>>>(xb, n, word);
   pa::quant::quantize_kernel<<<grid, pa::quant::kThreads, 0, s>>>(xb, n, word, static_cast<uint8_t*>(q));
-  pa::quant::scale_kernel<<<1, 1, 0, s>>>(word);
+  pa::quant::scale_kernel<<<1, 1, 0, s>>>(word, st->status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return PA_OK;
@@ -431,32 +467,12 @@ int pa_attn_fwd_chunks(const void* q, const void* const* k_chunks, const void* c
                        const int* nk_chunks, int n_chunks, void* o, float* lse, int B, int H, int Nq, int d,
                        float scale, void* stream) {
   g_err[0] = '\0';
-  if (!q || !k_chunks || !v_chunks || !nk_chunks || !o || !lse)
-    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
-  if (n_chunks < 1 || n_chunks > pa::single::kMaxChunks)
-    return fail(PA_ERR_INVALID_ARG, "n_chunks must be in [1, %d] (got %d)", pa::single::kMaxChunks, n_chunks);
   DeviceState* st = nullptr;
-  // Every chunk's host-side checks first, so no CUDA call is made for a bad table.
-  for (int pass = 0; pass < 2; ++pass)
-    for (int c = 0; c < n_chunks; ++c) {
-      const int rc = check_fwd_args(q, k_chunks[c], v_chunks[c], o, lse, B, H, Nq, nk_chunks[c], d, scale, &st,
-                                    pass == 0);
-      if (rc != PA_OK) return rc;
-    }
-  if (st == nullptr) return PA_OK;  // Nq == 0
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_fwd<64>(st, q, k_chunks, v_chunks, nk_chunks, n_chunks, o, lse, B * H, Nq, scale, s);
-  return launch_fwd<128>(st, q, k_chunks, v_chunks, nk_chunks, n_chunks, o, lse, B * H, Nq, scale, s);
-}
-
-int pa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
-                     int Nk, int d, float scale, void* stream) {
-  g_err[0] = '\0';
-  DeviceState* st = nullptr;
-  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, &st);
+  const int rc = check_chunk_args(q, k_chunks, v_chunks, nk_chunks, n_chunks, pa::single::kMaxChunks, o, lse, B, H,
+                                  Nq, d, scale, &st);
   if (rc != PA_OK || st == nullptr) return rc;
-  if (d != 128) return fail(PA_ERR_UNSUPPORTED, "d must be 128 for the CTA-pair kernel (got %d)", d);
-  return launch_fwd_pair(st, q, k, v, o, lse, B * H, Nq, Nk, scale, static_cast<cudaStream_t>(stream));
+  return launch_bf16(st, d, q, k_chunks, v_chunks, nk_chunks, n_chunks, o, lse, B * H, Nq, scale,
+                     static_cast<cudaStream_t>(stream));
 }
 
 int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void* o, float* lse, int B, int H,
@@ -512,19 +528,13 @@ int pa_attn_chunks_noalloc(const void* q, const void* const* k_chunks, const voi
     return fail(PA_ERR_INVALID_ARG, "the %d partial results need %llu bytes of scratch; the limit is %llu", n_chunks,
                 need, pa::kNoAllocScratchBytes);
   DeviceState* st = nullptr;
-  // Every chunk's host-side checks first, so no CUDA call is made for a bad table.
-  for (int pass = 0; pass < 2; ++pass)
-    for (int c = 0; c < n_chunks; ++c) {
-      const int rc = check_fwd_args(q, k_chunks[c], v_chunks[c], o, lse, B, H, Nq, nk_chunks[c], d, scale, &st,
-                                    pass == 0);
-      if (rc != PA_OK) return rc;
-    }
-  if (st == nullptr) return PA_OK;  // Nq == 0
+  const int rc0 = check_chunk_args(q, k_chunks, v_chunks, nk_chunks, n_chunks, pa::kNoAllocMaxChunks, o, lse, B, H,
+                                   Nq, d, scale, &st);
+  if (rc0 != PA_OK || st == nullptr) return rc0;  // st is null when Nq == 0
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int bh = B * H;
   auto fwd = [&](const void* k, const void* v, void* out, float* out_lse, int nk) {
-    return d == 64 ? launch_fwd<64>(st, q, &k, &v, &nk, 1, out, out_lse, bh, Nq, scale, s)
-                   : launch_fwd<128>(st, q, &k, &v, &nk, 1, out, out_lse, bh, Nq, scale, s);
+    return launch_bf16(st, d, q, &k, &v, &nk, 1, out, out_lse, bh, Nq, scale, s);
   };
   if (n_chunks == 1) return fwd(k_chunks[0], v_chunks[0], o, lse, nk_chunks[0]);
   // Every forward below writes its whole partial block before the merge reads
@@ -547,6 +557,7 @@ const char* pa_status_string(int code) {
     case PA_ERR_MISALIGNED: return "PA_ERR_MISALIGNED: pointer alignment";
     case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime or driver error";
     case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT: a device-side bounded wait gave up";
+    case PA_ERR_BAD_INPUT: return "PA_ERR_BAD_INPUT: a value read on the device was not finite or not positive";
     default: return "unknown status code";
   }
 }
@@ -587,6 +598,13 @@ int pa_selftest_timeout(int limit_us, void* stream) {
   return PA_OK;
 }
 
-int pa_version(void) { return 100; }
+int pa_set_wait_limit_ms(int ms) {
+  g_err[0] = '\0';
+  if (ms < 1 || ms > 600000) return fail(PA_ERR_INVALID_ARG, "ms must be in [1, 600000] (got %d)", ms);
+  g_wait_limit_ns.store(static_cast<unsigned long long>(ms) * 1000000ull, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+int pa_version(void) { return 200; }
 
 }  // extern "C"

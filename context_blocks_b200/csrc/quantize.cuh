@@ -10,7 +10,8 @@
 //   1. amax_kernel: |x| as bf16 bits (non-negative, so integer order is value
 //      order) reduced per warp and combined with atomicMax into the word;
 //   2. quantize_kernel: every block reads amax from the word, converts;
-//   3. scale_kernel: one thread replaces the word by the float scale.
+//   3. scale_kernel: one thread replaces the word by the float scale (and
+//      reports a non-finite amax in the device status word).
 // Both passes stream x with 16-byte loads (8 bf16); the second pass usually
 // hits L2 for inputs up to its size.
 #pragma once
@@ -18,6 +19,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "fwd_common.cuh"
 #include "ptx.cuh"
 
 namespace pa {
@@ -84,9 +86,12 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const __nv_bfloat16*
   }
 }
 
-__global__ void scale_kernel(unsigned* word) {
-  const float s = scale_from_word(*word);
-  *reinterpret_cast<float*>(word) = s;
+// A non-finite amax (an Inf or NaN element: bf16 magnitude bits >= 0x7F80)
+// leaves no usable scale; it is recorded in the device status word.
+__global__ void scale_kernel(unsigned* word, int* status) {
+  const unsigned w = *word;
+  if (w >= 0x7F80u) atomicCAS(status, 0, kStatusBadInput);
+  *reinterpret_cast<float*>(word) = scale_from_word(w);
 }
 
 }  // namespace quant

@@ -9,8 +9,9 @@
  *   pa_attn_merge  the exact combination of n such partial results, computed
  *                  over disjoint key chunks, into the full-sequence result.
  *
- * Around them: pa_attn_fwd_chunks (up to 8 chunks in one launch, no
- * partials), pa_attn_fwd_pair (the same forward on CTA pairs),
+ * Around them: pa_attn_fwd_accum (fold one chunk into a running fp32 O and
+ * LSE, the local step of a ring that receives chunks one at a time),
+ * pa_attn_fwd_chunks (up to 8 chunks in one launch, no partials),
  * pa_attn_fwd_fp8 / pa_attn_fwd_fp8_dev with pa_quantize_e4m3 (e4m3 inputs),
  * pa_attn_chunks_noalloc (chunks + merge with library-owned static scratch),
  * and the status helpers at the end of this file.
@@ -37,14 +38,16 @@
  *   Inputs and outputs must not overlap.
  * - q, k, v, o and o_parts must be 16-byte aligned (TMA / vector access);
  *   lse and lse_parts 4-byte aligned.
- * - d must be 64 or 128 (128 for the CTA-pair and e4m3 entry points).
+ * - d must be 64 or 128 (128 for the e4m3 entry points).
  * - `stream` is a cudaStream_t (0 = legacy default stream).  Calls are fully
  *   asynchronous: they validate arguments on the host, enqueue kernels on
  *   `stream` and return.  They never synchronise the host and never copy
  *   between host and device.
  * - Return values: PA_OK or a negative PA_ERR_* code for errors the host can
  *   see before or at launch.  Errors raised later on the device (a bounded
- *   wait that gave up) are reported by pa_poll_device_status().
+ *   wait that gave up, a bad value read on the device) are reported by
+ *   pa_poll_device_status(); the outputs of the work that raised one are
+ *   undefined.  A caller that needs to know polls after synchronising.
  */
 #ifndef PA_ATTN_H_
 #define PA_ATTN_H_
@@ -61,6 +64,12 @@ extern "C" {
 #define PA_ERR_MISALIGNED (-3)  /* a pointer breaks the alignment rule above */
 #define PA_ERR_CUDA (-4)        /* CUDA runtime / driver error; see pa_last_error() */
 #define PA_ERR_TIMEOUT (-5)     /* a device-side bounded wait gave up (from pa_poll_device_status) */
+#define PA_ERR_BAD_INPUT (-6)   /* a value read on the device (a dequantisation scale, a quantiser's
+                                   amax) was not finite or not positive (from pa_poll_device_status) */
+
+/* Flags of pa_attn_fwd_accum. */
+#define PA_ACCUM_FIRST 1 /* no incoming state: o_acc / lse_acc are only written */
+#define PA_ACCUM_FINAL 2 /* write the result as bf16 into o (and lse_acc), not into o_acc */
 
 /*
  * pa_attn_fwd - attention of Q against one K/V chunk.
@@ -87,6 +96,42 @@ extern "C" {
  */
 int pa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                 int Nq, int Nk, int d, float scale, void* stream);
+
+/*
+ * pa_attn_fwd_accum - fold the attention over one more K/V chunk into a
+ * running result.
+ *
+ * The step a device takes each time a block arrives on the ring (diffusers
+ * "Context parallelism", section "Ring Attention": attend with the block held,
+ * pass it on; once every block has been seen the result is the full-sequence
+ * attention).  The running state is the result over the chunks folded so far,
+ * kept in fp32: a normalised output o_acc and its natural-log LSE lse_acc.
+ * One call replaces it by the merge (as pa_attn_merge defines it) of that
+ * state with the attention of q over this chunk's keys:
+ *     o_acc, lse_acc  <-  merge((o_acc, lse_acc), attention(q, k, v))
+ * without rounding any partial output to bf16 and without a separate merge.
+ *
+ * q, k, v   as pa_attn_fwd (bf16, device, 16-byte aligned)           (input)
+ * o_acc     [B,H,Nq,d] fp32, device, 16-byte aligned     (state: read unless
+ *           PA_ACCUM_FIRST, written unless PA_ACCUM_FINAL)
+ * lse_acc   [B,H,Nq]   fp32, device, 4-byte aligned      (state: read unless
+ *           PA_ACCUM_FIRST, always written).  A row whose lse_acc is -inf
+ *           counts as empty (its o_acc row is not read).  Values must
+ *           otherwise be finite.
+ * o         [B,H,Nq,d] bf16, device, 16-byte aligned: with PA_ACCUM_FINAL
+ *           the final output goes here (and the final LSE to lse_acc);
+ *           without it o must be NULL
+ * flags     0, PA_ACCUM_FIRST, PA_ACCUM_FINAL or both (both = pa_attn_fwd
+ *           with the LSE written to lse_acc)
+ * B, H, Nq, Nk, d, scale, stream   as pa_attn_fwd
+ *
+ * The state is read and written in place, row by row, by the thread that
+ * owns the row; no other call may use it concurrently.  Errors: as
+ * pa_attn_fwd; PA_ERR_INVALID_ARG for unknown flags, a missing o with
+ * PA_ACCUM_FINAL or an o without it, and overlapping buffers.
+ */
+int pa_attn_fwd_accum(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, void* o,
+                      int B, int H, int Nq, int Nk, int d, float scale, int flags, void* stream);
 
 /*
  * pa_attn_fwd_fp8 - pa_attn_fwd with e4m3 (fp8) Q, K and V.
@@ -119,9 +164,10 @@ int pa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, 
  * read from device memory (each a float, e.g. written by pa_quantize_e4m3),
  * so that quantising and attending need no host synchronisation.
  *
- * q_scale, k_scale, v_scale   device pointers to one float each, 4-byte aligned,
- *                             finite and > 0 when the kernel runs (not checked:
- *                             they are read on the device)
+ * q_scale, k_scale, v_scale   device pointers to one float each, 4-byte aligned;
+ *                             read on the device, where a value that is not
+ *                             finite and > 0 raises PA_ERR_BAD_INPUT in the
+ *                             device status word (outputs then undefined)
  * everything else             as pa_attn_fwd_fp8
  *
  * Errors: as pa_attn_fwd_fp8; PA_ERR_INVALID_ARG for a null or host scale
@@ -151,8 +197,9 @@ int pa_attn_fwd_fp8_dev(const void* q, const void* k, const void* v, const float
  * n      >= 1
  *
  * Errors: PA_ERR_INVALID_ARG (null, n < 1, overlapping buffers, host memory),
- * PA_ERR_MISALIGNED, PA_ERR_CUDA.  Three kernels and one memset are enqueued
- * on `stream`; nothing is allocated.
+ * PA_ERR_MISALIGNED, PA_ERR_CUDA.  An Inf or NaN in x leaves no usable scale:
+ * it raises PA_ERR_BAD_INPUT in the device status word.  Three kernels and
+ * one memset are enqueued on `stream`; nothing is allocated.
  */
 int pa_quantize_e4m3(const void* x, long long n, void* q, float* scale, void* stream);
 
@@ -178,20 +225,6 @@ int pa_quantize_e4m3(const void* x, long long n, void* q, float* scale, void* st
 int pa_attn_fwd_chunks(const void* q, const void* const* k_chunks, const void* const* v_chunks,
                        const int* nk_chunks, int n_chunks, void* o, float* lse, int B, int H, int Nq, int d,
                        float scale, void* stream);
-
-/*
- * pa_attn_fwd_pair - pa_attn_fwd computed on pairs of CTAs.
- *
- * Same operation, arguments, layouts, ownership and errors as pa_attn_fwd
- * (diffusers "Context parallelism", section "Ring Attention"), for d = 128
- * only (PA_ERR_UNSUPPORTED otherwise).  Two CTAs of a thread-block cluster
- * share each tensor-core MMA (tcgen05 cta_group::2, M = 256), so each CTA
- * loads only half of every K and V tile.  Results agree with pa_attn_fwd
- * within rounding; which of the two is faster depends on the shape (the
- * benchmark reports both).
- */
-int pa_attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                     int Nq, int Nk, int d, float scale, void* stream);
 
 /*
  * pa_attn_merge - combine n partial results over disjoint key chunks.
@@ -262,11 +295,13 @@ const char* pa_last_error(void);
 
 /*
  * Read and clear the device status word of the current device.  Kernels set
- * it (first error wins) when a bounded wait inside them gives up; the kernel
- * then releases its resources and exits instead of hanging.  Returns PA_OK,
- * PA_ERR_TIMEOUT, or PA_ERR_CUDA if the word could not be read.  This call
- * synchronises with the device (it copies 4 bytes device -> host): call it
- * after the work of interest has completed, never on a hot path.
+ * it (first error wins) when a bounded wait inside them gives up (the kernel
+ * then releases its resources and exits instead of hanging; the outputs it
+ * did not write keep their old contents) or when they read a bad value.
+ * Returns PA_OK, PA_ERR_TIMEOUT, PA_ERR_BAD_INPUT, or PA_ERR_CUDA if the word
+ * could not be read.  This call synchronises with the device (it copies 4
+ * bytes device -> host): call it after the work of interest has completed,
+ * never on a hot path.
  */
 int pa_poll_device_status(void);
 
@@ -278,6 +313,15 @@ int pa_poll_device_status(void);
  * CUDA context stays usable.  Used by tests of the failure path.
  */
 int pa_selftest_timeout(int limit_us, void* stream);
+
+/*
+ * Limit of every device-side barrier wait, in milliseconds (1 .. 600000;
+ * default 5000), for launches made after the call, process-wide.  A wait that
+ * makes no progress for this long gives up and reports PA_ERR_TIMEOUT.  Raise
+ * it where the GPU is time-sliced among many processes and a kernel may be
+ * held off the GPU for long stretches.  Returns PA_OK or PA_ERR_INVALID_ARG.
+ */
+int pa_set_wait_limit_ms(int ms);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int pa_version(void);

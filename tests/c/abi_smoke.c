@@ -27,9 +27,10 @@ int main(void) {
   void* o = (void*)(a + 3 * mb);
   float* lse = (float*)(a + 4 * mb);
 
-  CHECK(pa_version() == 100);
+  CHECK(pa_version() == 200);
   CHECK(strcmp(pa_status_string(PA_OK), "PA_OK") == 0);
   CHECK(strncmp(pa_status_string(PA_ERR_TIMEOUT), "PA_ERR_", 7) == 0);
+  CHECK(strncmp(pa_status_string(PA_ERR_BAD_INPUT), "PA_ERR_", 7) == 0);
 
   CHECK(pa_attn_fwd(NULL, k, v, o, lse, 1, 1, 8, 8, 128, 0.125f, NULL) == PA_ERR_INVALID_ARG);
   CHECK(strlen(pa_last_error()) > 0);
@@ -52,6 +53,15 @@ int main(void) {
   CHECK(pa_attn_fwd_fp8(q, k, v, 1.0f, 1.0f, 1.0f, o, lse, 1, 1, 8, 8, 64, 0.125f, NULL) == PA_ERR_UNSUPPORTED);
   CHECK(pa_quantize_e4m3(q, 0, o, lse, NULL) == PA_ERR_INVALID_ARG);
   CHECK(pa_selftest_timeout(0, NULL) == PA_ERR_INVALID_ARG);
+  CHECK(pa_set_wait_limit_ms(0) == PA_ERR_INVALID_ARG);
+
+  /* accumulate: the final fold needs o, the others must not get one */
+  float* oacc = (float*)(a + 5 * mb);
+  CHECK(pa_attn_fwd_accum(q, k, v, oacc, lse, NULL, 1, 1, 8, 8, 128, 0.125f, PA_ACCUM_FINAL, NULL) ==
+        PA_ERR_INVALID_ARG);
+  CHECK(pa_attn_fwd_accum(q, k, v, oacc, lse, o, 1, 1, 8, 8, 128, 0.125f, PA_ACCUM_FIRST, NULL) ==
+        PA_ERR_INVALID_ARG);
+  CHECK(pa_attn_fwd_accum(q, k, v, oacc, lse, NULL, 1, 1, 0, 8, 128, 0.125f, 0, NULL) == PA_OK);
 
   if (failures) {
     fprintf(stderr, "%d check(s) failed\n", failures);

@@ -46,16 +46,22 @@ def test_status_codes_match_header():
     codes = {m.group(1): int(m.group(2)) for m in
              re.finditer(r"#define\s+(PA_\w+)\s+\(?(-?\d+)\)?", text)}
     for name in ("PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_MISALIGNED",
-                 "PA_ERR_CUDA", "PA_ERR_TIMEOUT"):
+                 "PA_ERR_CUDA", "PA_ERR_TIMEOUT", "PA_ERR_BAD_INPUT", "PA_ACCUM_FIRST", "PA_ACCUM_FINAL"):
         assert codes[name] == getattr(B, name), name
 
 
 def test_status_strings(lib):
     assert B.status_string(0) == "PA_OK"
-    for code in (-1, -2, -3, -4, -5):
+    for code in (-1, -2, -3, -4, -5, -6):
         assert B.status_string(code).startswith("PA_ERR_")
     assert B.status_string(12345) == "unknown status code"
-    assert B.version() == 100
+    assert B.version() == 200
+
+
+def test_wait_limit_setter(lib):
+    assert lib.pa_set_wait_limit_ms(0) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_set_wait_limit_ms(600001) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_set_wait_limit_ms(5000) == B.PA_OK
 
 
 A = 1 << 20          # a 16-byte aligned fake address; never dereferenced
@@ -136,12 +142,24 @@ def test_build_flags_target_sm100a():
     assert "arch=compute_100a,code=sm_100a" in build_mod.NVCC_FLAGS
 
 
-def test_pair_argument_checks(lib):
-    f = lib.pa_attn_fwd_pair
-    assert f(0, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 128, 0.1, None) == B.PA_ERR_INVALID_ARG
-    assert f(A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 96, 0.1, None) == B.PA_ERR_UNSUPPORTED
-    assert f(A + 8, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 8, 8, 128, 0.1, None) == B.PA_ERR_MISALIGNED
-    assert f(A, A + MB, A + 2 * MB, A + 3 * MB, A + 4 * MB, 1, 1, 0, 8, 128, 0.1, None) == B.PA_OK
+def _accum(lib, q=A, k=A + MB, v=A + 2 * MB, oacc=A + 5 * MB, lacc=A + 4 * MB, o=0, Nq=8, Nk=8, d=128,
+           flags=0):
+    return lib.pa_attn_fwd_accum(q, k, v, oacc, lacc, o or None, 1, 1, Nq, Nk, d, 0.125, flags, None)
+
+
+def test_accum_argument_checks(lib):
+    assert _accum(lib, q=0) == B.PA_ERR_INVALID_ARG
+    assert _accum(lib, oacc=0) == B.PA_ERR_INVALID_ARG
+    assert _accum(lib, flags=4) == B.PA_ERR_INVALID_ARG                       # unknown flag
+    assert _accum(lib, flags=B.PA_ACCUM_FINAL) == B.PA_ERR_INVALID_ARG        # final fold without o
+    assert _accum(lib, o=A + 3 * MB) == B.PA_ERR_INVALID_ARG                  # o without the final fold
+    assert _accum(lib, d=96) == B.PA_ERR_UNSUPPORTED
+    assert _accum(lib, oacc=A + 5 * MB + 8) == B.PA_ERR_MISALIGNED
+    assert _accum(lib, oacc=A + 2 * MB + 64) == B.PA_ERR_INVALID_ARG          # state inside v
+    # the fp32 state is 4 bytes per element: 8 rows x 128 x 4 = 4 KB past o_acc
+    assert _accum(lib, lacc=A + 5 * MB + 4096 - 4) == B.PA_ERR_INVALID_ARG
+    assert _accum(lib, o=A + 5 * MB + 1024, flags=B.PA_ACCUM_FINAL) == B.PA_ERR_INVALID_ARG  # o inside the state
+    assert _accum(lib, Nq=0, flags=B.PA_ACCUM_FIRST) == B.PA_OK
 
 
 def _chunks(lib, n=3, nk=(8, 8, 8), kaddr=None, Nq=8, d=128, q=A, o=A + 3 * MB, lse=A + 4 * MB):

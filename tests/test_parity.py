@@ -500,58 +500,48 @@ def test_fp8_rejects_bf16(pa):
         pa.attn_fwd_fp8(q, q, q, 1.0, 1.0, 1.0)
 
 
-# ---------------------------------------------------------------- CTA-pair kernel
+# ---------------------------------------------------------------- values read on the device
 
-def _pair_case(pa, q, k, v, scale, what):
-    o = torch.full_like(q, float("nan"))
-    lse = torch.full(q.shape[:3], float("nan"), device="cuda")
-    pa.attn_fwd(q, k, v, scale=scale, out=o, lse=lse, pair=True)
+def test_fp8_device_scale_that_is_not_positive_is_reported(pa):
+    """A dequantisation scale read on the device that is zero, negative, Inf
+    or NaN is recorded as PA_ERR_BAD_INPUT in the status word (a normal
+    launch: the kernel runs to the end, its outputs are meaningless)."""
+    w = workloads.Workload("badscale", B=1, H=1, Nq=128, Nk=256, d=128, rms_qk=True, chunks=(256,), seed=63)
+    q, k, v = workloads.make_case(w, device="cuda")
+    (q8, sq), (k8, sk), (v8, sv) = pa.quantize_e4m3(q), pa.quantize_e4m3(k), pa.quantize_e4m3(v)
     torch.cuda.synchronize()
     assert pa.poll_device_status() == pa.PA_OK
-    o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), scale)
-    assert_close(o, lse, o_ref, l_ref, what)
-    return o, lse
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        for which in range(3):
+            scales = [sq.clone(), sk.clone(), sv.clone()]
+            scales[which].fill_(bad)
+            pa.attn_fwd_fp8(q8, k8, v8, *scales, scale=w.scale)
+            torch.cuda.synchronize()
+            assert pa.poll_device_status() == pa.PA_ERR_BAD_INPUT, (bad, which)
+    # good scales again: clean status, correct result
+    o, lse = pa.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, scale=w.scale, check=True)
+    qd, kd, vd = (_dequant(a, float(b.item())) for a, b in ((q8, sq), (k8, sk), (v8, sv)))
+    o_ref, l_ref = oracle.attention(qd, kd, vd, w.scale)
+    assert_close_fp8(o, lse, o_ref, l_ref, float(vd.abs().max()), "fp8 after bad scales")
 
 
-def test_pair_flux(pa):
-    w = workloads.get("flux")
+def test_quantize_reports_non_finite_input(pa):
+    for bad in (float("inf"), float("-inf"), float("nan")):
+        x = torch.randn((4099,), device="cuda").to(torch.bfloat16)
+        x[1234] = bad
+        pa.quantize_e4m3(x)
+        torch.cuda.synchronize()
+        assert pa.poll_device_status() == pa.PA_ERR_BAD_INPUT, bad
+        # the binding's check option raises on the same condition
+        with pytest.raises(pa.PaError) as e:
+            pa.quantize_e4m3(x, check=True)
+        assert e.value.code == pa.PA_ERR_BAD_INPUT
+        assert pa.poll_device_status() == pa.PA_OK     # the check consumed the status
+
+
+def test_check_option_passes_on_good_input(pa):
+    w = workloads.get("tiny")
     q, k, v = workloads.make_case(w, device="cuda")
-    o, lse = _pair_case(pa, q, k, v, w.scale, "pair flux")
-    o1, l1 = pa.attn_fwd(q, k, v, scale=w.scale)
-    torch.cuda.synchronize()
-    # the two kernels compute the same values in the same order per row
-    assert (o.float() - o1.float()).abs().max().item() <= 2 ** -8
-    assert (lse - l1).abs().max().item() <= 1e-5
-
-
-def test_pair_uneven_tail_chunk(pa):
-    w = workloads.get("tails")
-    q, k, v = workloads.make_case(w, device="cuda")
-    _pair_case(pa, q, k[:, :, :1151].contiguous(), v[:, :, :1151].contiguous(), w.scale, "pair tails chunk")
-
-
-@pytest.mark.parametrize("B,H,Nq,Nk,d", [e for e in EDGE if e[4] == 128])
-def test_pair_edge_shapes(pa, B, H, Nq, Nk, d):
-    g = torch.Generator(device="cuda").manual_seed(2000 + Nq * 7 + Nk * 13)
-    q = torch.randn((B, H, Nq, d), generator=g, device="cuda").to(torch.bfloat16)
-    k = torch.randn((B, H, Nk, d), generator=g, device="cuda").to(torch.bfloat16)
-    v = torch.randn((B, H, Nk, d), generator=g, device="cuda").to(torch.bfloat16)
-    _pair_case(pa, q, k, v, 1.0 / math.sqrt(d), f"pair edge {(B, H, Nq, Nk, d)}")
-
-
-def test_pair_rescale_path(pa):
-    B, H, Nq, Nk, d = 1, 2, 600, 1100, 128
-    g = torch.Generator(device="cuda").manual_seed(81)
-    q = torch.randn((B, H, Nq, d), generator=g, device="cuda") * 0.2 + 1.0
-    ramp = torch.linspace(0.0, 1.0, Nk, device="cuda")[None, None, :, None]
-    k = torch.randn((B, H, Nk, d), generator=g, device="cuda") * 0.1 + ramp * 6.0
-    v = torch.randn((B, H, Nk, d), generator=g, device="cuda")
-    q, k, v = (x.to(torch.bfloat16).contiguous() for x in (q, k, v))
-    _pair_case(pa, q, k, v, 1.0 / math.sqrt(d), "pair rising logits")
-
-
-def test_pair_rejects_head_dim_64(pa):
-    q = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(pa.PaError) as e:
-        pa.attn_fwd(q, q.clone(), q.clone(), pair=True)
-    assert e.value.code == pa.PA_ERR_UNSUPPORTED
+    o, lse = pa.attn_fwd(q, k, v, scale=w.scale, check=True)
+    o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), w.scale)
+    assert_close(o, lse, o_ref, l_ref, "attn_fwd with check=True")

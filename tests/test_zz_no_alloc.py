@@ -5,11 +5,15 @@ under a framework's allocator, loops that cannot afford cudaMalloc's
 device-wide synchronisation, plug-ins handed only their inputs and outputs).
 For them the library keeps the per-chunk partial results in one static
 device array instead of buffers someone allocates.  These tests call that
-entry point through the C ABI and hold its output against the existing entry
-points (pa_attn_fwd per chunk into caller-allocated partials, then
-pa_attn_merge), within the parity tolerances, on two calls in a row with
-different inputs: the shared array still holds the first call's partials when
-the second call runs.  A shape whose partials do not fit is refused.
+entry point through the C ABI and hold its output both against the fp64
+oracle over the unchunked keys and against the existing entry points
+(pa_attn_fwd per chunk into caller-allocated partials, then pa_attn_merge),
+within the parity tolerances, on two calls in a row with different inputs:
+the shared array still holds the first call's partials when the second call
+runs.  A larger call followed by a smaller one with a different chunk count
+checks that stale partials at other offsets are never read, and one case goes
+through the Python binding with caller-supplied outputs.  A shape whose
+partials do not fit is refused.
 
 This file is collected last, so a run that stops at the first failure has
 already run every other test.
@@ -22,6 +26,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
 from tests._parity import assert_close
 
@@ -63,13 +68,15 @@ def _check_against_existing(pa, w, seed):
     q, k, v = workloads.make_case(w, device="cuda", seed=seed)
     pairs = workloads.split_keys(k, v, w.chunks)
     kc, vc = [p[0] for p in pairs], [p[1] for p in pairs]
-    o_ref, l_ref = _existing(pa, q, kc, vc, w.scale)
+    o_ex, l_ex = _existing(pa, q, kc, vc, w.scale)
     rc, o, lse = _noalloc_c_abi(pa, q, kc, vc, w.scale)
     assert rc == pa.PA_OK, pa.last_error()
     torch.cuda.synchronize()
     assert pa.poll_device_status() == pa.PA_OK
-    assert_close(o, lse, o_ref.float().cpu().double().numpy(), l_ref.cpu().double().numpy(),
+    assert_close(o, lse, o_ex.float().cpu().double().numpy(), l_ex.cpu().double().numpy(),
                  f"no-alloc vs existing entry points ({w.name}, seed {seed})")
+    o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), w.scale)
+    assert_close(o, lse, o_ref, l_ref, f"no-alloc vs oracle over all keys ({w.name}, seed {seed})")
     return o, lse
 
 
@@ -85,6 +92,39 @@ def test_noalloc_uneven_chunks_head_dim_64(pa):
                            chunks=(200, 1, 316), seed=7)
     _check_against_existing(pa, w, seed=7)
     _check_against_existing(pa, w, seed=8)
+
+
+def test_noalloc_larger_call_then_smaller_call(pa):
+    """8 chunks fill most of the array; then 3 chunks of another shape place
+    their partials at other offsets, over what the first call left."""
+    big = workloads.Workload("noalloc_big", B=1, H=8, Nq=1000, Nk=8 * 150, d=128, rms_qk=True,
+                             chunks=(150,) * 8, seed=9)
+    small = workloads.Workload("noalloc_small", B=2, H=2, Nq=333, Nk=401, d=128, rms_qk=False,
+                               chunks=(129, 255, 17), seed=10)
+    _check_against_existing(pa, big, seed=11)
+    _check_against_existing(pa, small, seed=12)
+    _check_against_existing(pa, big, seed=13)
+
+
+def test_noalloc_through_the_binding(pa):
+    """The public binding with caller-supplied outputs, and its shape checks."""
+    w = workloads.get("flux1008")
+    q, k, v = workloads.make_case(w, device="cuda", seed=14)
+    q = q[:, :4].contiguous()                     # 4 heads: partials fit the array
+    pairs = workloads.split_keys(k[:, :4].contiguous(), v[:, :4].contiguous(), w.chunks)
+    kc, vc = [p[0] for p in pairs], [p[1] for p in pairs]
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:3], float("nan"), dtype=torch.float32, device="cuda")
+    o2, l2 = pa.attn_chunks_noalloc(q, kc, vc, scale=w.scale, out=o, lse=lse, check=True)
+    assert o2.data_ptr() == o.data_ptr() and l2.data_ptr() == lse.data_ptr()
+    kh = torch.cat([a.cpu() for a in kc], dim=2)
+    vh = torch.cat([b.cpu() for b in vc], dim=2)
+    o_ref, l_ref = oracle.attention(q.cpu(), kh, vh, w.scale)
+    assert_close(o, lse, o_ref, l_ref, "no-alloc through the binding")
+    with pytest.raises(ValueError):
+        pa.attn_chunks_noalloc(q, kc, vc, out=torch.empty((1, 4, 7, 128), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        pa.attn_chunks_noalloc(q, kc, vc, lse=torch.empty((1, 4, w.Nq), dtype=torch.float64, device="cuda"))
 
 
 def test_noalloc_single_chunk(pa):
