@@ -1,0 +1,209 @@
+"""Context parallelism across GPUs: the ring of K/V blocks and the Ulysses
+all-to-all, each around the library's single-GPU kernels.
+
+Both follow the diffusers guide "Context parallelism":
+
+* section "Ring Attention": every device holds one block of the sequence's
+  queries, keys and values.  At each step it attends with the K/V block it
+  currently holds and passes that block to the next device, receiving the
+  previous device's; after as many steps as there are devices it has seen
+  every block, and its queries' attention is exact.  Here each step folds
+  the block into a running fp32 (O, LSE) with ``pa_attn_fwd_accum``, and the
+  transfer of the next block runs on a separate CUDA stream while the fold
+  runs, into one of two receive buffers in local HBM (a remote block is
+  always copied into this GPU's memory before a kernel reads it).
+  Blocks may differ in length (section "Ring Anything Attention": each block
+  keeps its real length; padding never enters the softmax).
+* section "Ulysses Attention": an all-to-all turns sequence-sharded Q, K, V
+  into head-sharded tensors over the whole sequence, each device attends for
+  its heads with ``pa_attn_fwd``, and a second all-to-all turns the output
+  back.  It needs the head count, and the per-device sequence length, to be
+  the same on every device and the heads to divide by the device count.
+
+The functions take a ``torch.distributed`` process group (NCCL for CUDA
+tensors).  The arithmetic of a step is passed in as ``attend`` /
+``attend_full`` so that the exchange schedule can be exercised with CPU
+tensors and the gloo backend; by default it is the library's kernels.
+"""
+
+from __future__ import annotations
+
+from typing import Callable, List, Optional, Sequence
+
+__all__ = ["ring_schedule", "ring_attention", "ulysses_attention"]
+
+
+def ring_schedule(rank: int, world: int) -> List[dict]:
+    """Which block rank `rank` attends to at each step, and who it sends to
+    and receives from (blocks are named by the rank that owns them).
+
+    Step s: attend to the block of rank (rank - s) mod world, send it to
+    (rank + 1) mod world and, except on the last step, receive the block of
+    rank (rank - s - 1) mod world from (rank - 1) mod world into receive
+    buffer s mod 2.  Step s + 1 attends to that buffer; the block of step 0
+    is the rank's own."""
+    out = []
+    for s in range(world):
+        ent = {"step": s, "block": (rank - s) % world, "buffer": None if s == 0 else (s - 1) % 2}
+        if s < world - 1:
+            ent.update(send_to=(rank + 1) % world, recv_from=(rank - 1) % world,
+                       recv_block=(rank - s - 1) % world, recv_buffer=s % 2)
+        out.append(ent)
+    return out
+
+
+def _default_attend(q, k, v, o_acc, lse_acc, first, final, out, scale):
+    from ._binding import attn_fwd_accum
+    attn_fwd_accum(q, k, v, o_acc, lse_acc, first=first, final=final, out=out, scale=scale)
+
+
+def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None, scale: Optional[float] = None,
+                   out=None, attend: Optional[Callable] = None, comm_stream=None, trace: Optional[list] = None):
+    """Ring attention of this rank's queries over every rank's K/V block.
+
+    q [B,H,n_q,d] and k, v [B,H,n_kv,d] are this rank's blocks (bf16 CUDA
+    tensors for the library's kernels).  ``kv_lens`` lists every rank's K/V
+    block length (gathered from the ranks when not given).  Returns
+    (o [B,H,n_q,d], lse [B,H,n_q] fp32): this rank's queries attended over
+    the whole sequence.  ``trace``, if a list, receives one entry per step
+    (the schedule as executed)."""
+    import math
+
+    import torch
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, H, n_q, d = q.shape
+    if k.shape != v.shape or tuple(k.shape[:2]) != (B, H) or k.shape[3] != d:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    attend = attend or _default_attend
+    if kv_lens is None:
+        n = torch.tensor([k.shape[2]], dtype=torch.int64, device=q.device)
+        lens = [torch.zeros_like(n) for _ in range(world)]
+        dist.all_gather(lens, n, group=group)
+        kv_lens = [int(x.item()) for x in lens]
+    kv_lens = [int(x) for x in kv_lens]
+    if len(kv_lens) != world or kv_lens[rank] != k.shape[2] or min(kv_lens) < 1:
+        raise ValueError(f"kv_lens {kv_lens} does not match the group ({world} ranks, own block {k.shape[2]})")
+
+    cuda = q.is_cuda
+    o_acc = torch.empty((B, H, n_q, d), dtype=torch.float32, device=q.device)
+    lse_acc = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if world == 1:
+        attend(q, k, v, o_acc, lse_acc, True, True, out, scale)
+        if trace is not None:
+            trace.append({"step": 0, "block": 0})
+        return out, lse_acc
+
+    # Two receive buffers, each big enough for the longest block.
+    m = max(kv_lens)
+    bufs = [(torch.empty(B * H * m * d, dtype=k.dtype, device=k.device),
+             torch.empty(B * H * m * d, dtype=v.dtype, device=v.device)) for _ in range(2)]
+
+    def view(buf, n):
+        return buf[:B * H * n * d].view(B, H, n, d)
+
+    compute = torch.cuda.current_stream(q.device) if cuda else None
+    comm = (comm_stream or torch.cuda.Stream(device=q.device)) if cuda else None
+    if cuda:
+        comm.wait_stream(compute)          # the own block (and q) are ready
+    cur_k, cur_v = k, v
+    recv_done = None
+    prev_compute_done = None
+    sched = ring_schedule(rank, world)
+    for s, ent in enumerate(sched):
+        reqs = []
+        nxt = None
+        if s < world - 1:
+            nb = kv_lens[ent["recv_block"]]
+            nxt = (view(bufs[ent["recv_buffer"]][0], nb), view(bufs[ent["recv_buffer"]][1], nb))
+            ops = [dist.P2POp(dist.isend, cur_k, ent["send_to"], group),
+                   dist.P2POp(dist.isend, cur_v, ent["send_to"], group),
+                   dist.P2POp(dist.irecv, nxt[0], ent["recv_from"], group),
+                   dist.P2POp(dist.irecv, nxt[1], ent["recv_from"], group)]
+            if cuda:
+                with torch.cuda.stream(comm):
+                    # The buffer being received into held the block of step
+                    # s - 1: its fold must be done before it is overwritten.
+                    if prev_compute_done is not None:
+                        comm.wait_event(prev_compute_done)
+                    reqs = dist.batch_isend_irecv(ops)
+                    for r in reqs:
+                        r.wait()           # makes the comm stream wait for the transfer
+                    recv_done = torch.cuda.Event()
+                    recv_done.record(comm)
+            else:
+                reqs = dist.batch_isend_irecv(ops)
+        attend(q, cur_k, cur_v, o_acc, lse_acc, s == 0, s == world - 1, out if s == world - 1 else None, scale)
+        if trace is not None:
+            trace.append({"step": s, "block": ent["block"], "n_keys": int(cur_k.shape[2])})
+        if s < world - 1:
+            if cuda:
+                prev_compute_done = torch.cuda.Event()
+                prev_compute_done.record(compute)
+                compute.wait_event(recv_done)
+            else:
+                for r in reqs:
+                    r.wait()
+            cur_k, cur_v = nxt
+    if cuda:
+        # Work after this call (and the receive buffers' release) comes after
+        # everything the comm stream did.
+        compute.wait_stream(comm)
+    return out, lse_acc
+
+
+def _a2a(x, group):
+    """all_to_all over dim 0 of a contiguous tensor (one slice per rank)."""
+    import torch
+    import torch.distributed as dist
+    y = torch.empty_like(x)
+    dist.all_to_all_single(y, x, group=group)
+    return y
+
+
+def _default_attend_full(q, k, v, scale):
+    from ._binding import attn_fwd
+    return attn_fwd(q, k, v, scale=scale)
+
+
+def ulysses_attention(q, k, v, group=None, scale: Optional[float] = None, attend_full: Optional[Callable] = None):
+    """Ulysses attention: this rank's sequence shard q, k, v [B,H,n,d] (the
+    same n and H on every rank, H divisible by the rank count) in, this
+    rank's shard of the output (o [B,H,n,d], lse [B,H,n] fp32) out."""
+    import math
+
+    import torch
+    import torch.distributed as dist
+
+    P = dist.get_world_size(group)
+    B, H, n, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("Ulysses needs q, k, v of one shape [B,H,n,d] on every rank")
+    if H % P:
+        raise ValueError(f"{H} heads do not divide over {P} ranks")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    attend_full = attend_full or _default_attend_full
+    Hp = H // P
+
+    def to_heads(x):
+        # [B, H, n, d] -> send head group j to rank j -> [B, Hp, P*n, d] (sequence in rank order)
+        xs = x.reshape(B, P, Hp, n, *x.shape[3:]).transpose(0, 1).contiguous()
+        y = _a2a(xs, group)                                      # [P(src rank), B, Hp, n, ...]
+        return y.permute(1, 2, 0, *range(3, y.dim())).reshape(B, Hp, P * n, *x.shape[3:]).contiguous()
+
+    def to_seq(y):
+        # [B, Hp, P*n, ...] -> back to [B, H, n, ...] for this rank's sequence shard
+        ys = y.reshape(B, Hp, P, n, *y.shape[3:]).permute(2, 0, 1, *range(3, y.dim() + 1)).contiguous()
+        z = _a2a(ys, group)                                      # [P(src head group), B, Hp, n, ...]
+        return z.transpose(0, 1).reshape(B, H, n, *y.shape[3:]).contiguous()
+
+    qh, kh, vh = to_heads(q), to_heads(k), to_heads(v)
+    o_h, lse_h = attend_full(qh, kh, vh, scale)
+    return to_seq(o_h), to_seq(lse_h)

@@ -1,0 +1,157 @@
+"""The multi-rank exchange schedules of context_parallel on the CPU: gloo
+process groups of 2 and 3 ranks, float64 tensors, and the attention step
+injected by the test (the fp64 oracle), so that what is checked here is the
+exchange itself: which block each rank folds at each step, from which
+buffer, that the ring's blocks may differ in length, and that both the ring
+and the Ulysses all-to-all give every rank exactly the attention of its
+queries over the whole sequence (diffusers "Context parallelism", sections
+"Ring Attention", "Ring Anything Attention" and "Ulysses Attention")."""
+
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from context_blocks_b200.context_parallel import ring_schedule
+
+SCALE = 0.3
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _global_case(seed, B, H, n_total, d):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, H, n_total, d), generator=g, dtype=torch.float64)
+    k = torch.randn((B, H, n_total, d), generator=g, dtype=torch.float64)
+    v = torch.randn((B, H, n_total, d), generator=g, dtype=torch.float64)
+    return q, k, v
+
+
+def _oracle_fold(q, k, v, o_acc, lse_acc, first, final, out, scale):
+    """The fold of one block, from the oracle: merge the running state with
+    the attention over this block."""
+    o_b, l_b = oracle.attention(q, k, v, scale)
+    if first:
+        o_new, l_new = o_b, l_b
+    else:
+        o_new, l_new = oracle.merge(np.stack([o_acc.numpy(), o_b]), np.stack([lse_acc.numpy(), l_b]))
+    lse_acc.copy_(torch.from_numpy(l_new))
+    (out if final else o_acc).copy_(torch.from_numpy(o_new))
+
+
+def _ring_rank(rank, world, port, q_lens, kv_lens, gather, out_q):
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import ring_attention
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        q, k, v = _global_case(5, 2, 3, max(sum(q_lens), sum(kv_lens)), 8)
+        qs = np.cumsum([0] + list(q_lens))
+        ks = np.cumsum([0] + list(kv_lens))
+        q_r = q[:, :, qs[rank]:qs[rank + 1]].contiguous()
+        k_r = k[:, :, ks[rank]:ks[rank + 1]].contiguous()
+        v_r = v[:, :, ks[rank]:ks[rank + 1]].contiguous()
+        trace = []
+        passed = None if gather else kv_lens   # None: the ranks gather the lengths themselves
+        o = torch.empty(q_r.shape, dtype=torch.float64)
+        lse = torch.empty(q_r.shape[:3], dtype=torch.float64)
+
+        def attend(qq, kk, vv, o_acc, lse_acc, first, final, out, scale):
+            # the driver's running state is float32 for the kernels; here it is
+            # replaced by float64 buffers of the same shape
+            _oracle_fold(qq, kk, vv, o, lse, first, final, out, scale)
+
+        out, _ = ring_attention(q_r, k_r, v_r, kv_lens=passed, scale=SCALE, out=torch.empty_like(q_r),
+                                attend=attend, trace=trace)
+        o_ref, l_ref = oracle.attention(q_r, k[:, :, :ks[-1]], v[:, :, :ks[-1]], SCALE)
+        out_q.put((rank, float(np.abs(out.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()),
+                   trace))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _run(target, world, *args):
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=target, args=(r, world, port, *args, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        r = q.get(timeout=180)
+        got[r[0]] = r[1:]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return got
+
+
+def test_ring_schedule_visits_every_block_once():
+    for world in (1, 2, 3, 4, 8):
+        for rank in range(world):
+            sched = ring_schedule(rank, world)
+            assert [e["block"] for e in sched] == [(rank - s) % world for s in range(world)]
+            assert sorted(e["block"] for e in sched) == list(range(world))
+            for s, e in enumerate(sched[:-1]):
+                # what is received at step s is what step s + 1 folds, from
+                # the buffer the receive wrote
+                assert e["recv_block"] == sched[s + 1]["block"]
+                assert e["recv_buffer"] == sched[s + 1]["buffer"]
+                # the previous rank holds that block at step s
+                assert ring_schedule(e["recv_from"], world)[s]["block"] == e["recv_block"]
+                assert ring_schedule(e["send_to"], world)[s]["recv_from"] == rank
+            # a receive never overwrites the buffer folded at the same step
+            for e in sched[1:-1]:
+                assert e["recv_buffer"] != e["buffer"]
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,gather", [((6, 6), (6, 6), False), ((5, 9, 4), (7, 3, 11), True)])
+def test_ring_attention_gloo(q_lens, kv_lens, gather):
+    world = len(q_lens)
+    got = _run(_ring_rank, world, q_lens, kv_lens, gather)
+    for rank in range(world):
+        err_o, err_l, trace = got[rank]
+        assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
+        assert [t["block"] for t in trace] == [(rank - s) % world for s in range(world)]
+        assert [t["n_keys"] for t in trace] == [kv_lens[(rank - s) % world] for s in range(world)]
+
+
+def _ulysses_rank(rank, world, port, n, H, out_q):
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import ulysses_attention
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        q, k, v = _global_case(6, 2, H, n * world, 8)
+        sl = slice(rank * n, (rank + 1) * n)
+        seen = []
+
+        def attend_full(qh, kh, vh, scale):
+            seen.append(tuple(qh.shape))
+            o, l = oracle.attention(qh, kh, vh, scale)
+            return torch.from_numpy(o), torch.from_numpy(l)
+
+        o, lse = ulysses_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
+                                   scale=SCALE, attend_full=attend_full)
+        o_ref, l_ref = oracle.attention(q[:, :, sl], k, v, SCALE)
+        out_q.put((rank, float(np.abs(o.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()), seen))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,H", [(2, 4), (3, 6)])
+def test_ulysses_attention_gloo(world, H):
+    n = 5
+    got = _run(_ulysses_rank, world, n, H)
+    for rank in range(world):
+        err_o, err_l, seen = got[rank]
+        assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
+        assert seen == [(2, H // world, n * world, 8)]     # its heads, the whole sequence
