@@ -1,19 +1,26 @@
 """Benchmark of the blockwise attention library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload flux] [--no-extra] [--no-cpu-baseline]
+                    [--workload hunyuan] [--no-extra] [--no-cpu-baseline]
 
 One step is one pass of the hot path over one batch of the named workload:
 ``pa_attn_fwd`` over each K/V chunk, then ``pa_attn_merge`` when the workload
-has more than one chunk.  The default workload is the FLUX-shaped joint
-attention (B=1, H=24, Nq=Nk=4608, d=128, one chunk).  The metric is attention
-forward TFLOPS, 4*B*H*Nq*Nk*d per step over the device time.
+has more than one chunk.  The default workload is the largest one-GPU
+configuration, the HunyuanVideo-shaped attention (B=1, H=24,
+Nq=Nk=119056, d=128, one chunk); the FLUX-shaped one is reported among the
+extras.  The metric is attention forward TFLOPS, 4*B*H*Nq*Nk*d per step over
+the device time.
 
-Multi-GPU: one process per GPU (torchrun), every rank runs an independent
-replica of the step (the attention calls of different heads, batches or
-query blocks share nothing), so scaling is weak and there is no data-path
-collective; the process group only provides the barrier and the max over
-ranks of the timed region.
+Multi-GPU: one process per GPU (torchrun).  By default (``--parallel ring``)
+the ranks run Ring Attention over the named workload (diffusers "Context
+parallelism", section "Ring Attention"): each rank holds 1/N of the query
+rows and of the K/V rows, folds each K/V block into its running state with
+``pa_attn_fwd_accum`` while the next block arrives from the previous rank
+over NCCL on a second stream.  The whole problem is fixed as N grows, so
+scaling is strong.  ``--parallel replicas`` runs an independent copy of the
+single-GPU step on every rank instead (weak scaling, no data-path
+collective).  Either way the process group provides the barrier and the max
+over ranks of the timed region.
 
 Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
 on a bounded sample of the same workload instead (the reference arm).
@@ -101,7 +108,7 @@ class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML (read only)
     from a thread while the timed region runs."""
 
-    def __init__(self, torch_device: int, period_s: float = 0.02):
+    def __init__(self, torch_device: int, period_s: float = 0.005):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
@@ -187,10 +194,9 @@ def aggregate_throughput(flops_per_step_per_rank: float, steps: int, world: int,
 class Step:
     """Buffers and launches of one hot-path step on one workload."""
 
-    def __init__(self, w: workloads.Workload, sets: int, device, pair: bool = False, fp8: bool = False, pa=None):
+    def __init__(self, w: workloads.Workload, sets: int, device, fp8: bool = False, pa=None):
         import torch
         self.w = w
-        self.pair = pair
         self.fp8 = fp8
         self.sets = []
         n = len(w.chunks)
@@ -246,7 +252,7 @@ class Step:
             ls = lse if n == 1 else lse_parts[p]
             if fwd_events is not None:
                 fwd_events[0].append(_record())
-            pa.attn_fwd(q, k, v, scale=self.w.scale, out=out, lse=ls, pair=self.pair)
+            pa.attn_fwd(q, k, v, scale=self.w.scale, out=out, lse=ls)
             if fwd_events is not None:
                 fwd_events[1].append(_record())
         if n > 1:
@@ -271,11 +277,11 @@ def _sets_for(w: workloads.Workload, fp8: bool = False) -> int:
     return max(1, min(8, math.ceil(2.5 * L2_BYTES / per_set)))
 
 
-def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, pair=False, fp8=False):
+def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, fp8=False):
     """Device time of `steps` steps (CUDA events on the launching stream,
     synchronised on both sides).  Returns a dict of timings."""
     import torch
-    st = Step(w, _sets_for(w, fp8), device, pair=pair, fp8=fp8, pa=pa)
+    st = Step(w, _sets_for(w, fp8), device, fp8=fp8, pa=pa)
     for i in range(warmup):
         st.run(i, pa)
     torch.cuda.synchronize()
@@ -447,11 +453,11 @@ def oracle_sample(w, seconds: float, seed_rows: int = 0):
 
 # --------------------------------------------------------------------- main
 
-def _config(w, sets=None, resident_mb=None):
+def _config(w, sets=None, resident_mb=None, parallelism="one GPU"):
     c = {"workload": f"{w.name}: B={w.B} H={w.H} Nq={w.Nq} Nk={w.Nk} d={w.d}, "
                      f"{len(w.chunks)} K/V chunk(s) {list(w.chunks) if len(w.chunks) > 1 else ''}".strip(),
          "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "chunks": list(w.chunks),
-         "parallelism": "replicas (one independent step per GPU)"}
+         "parallelism": parallelism}
     if sets is not None:
         c["l2"] = (f"inputs rotate over {sets} seeded sets, {resident_mb:.0f} MB resident "
                    f"> 126 MB L2, so no step reads the previous step's inputs from L2")
@@ -523,6 +529,8 @@ def run_ours(args):
     peaks = _peaks()
     sampler = ClockSampler(local)
     fp8 = bool(getattr(args, "fp8", False))
+    if ws > 1 and args.parallel == "ring":
+        return run_ring(args, pa, w, peaks, sampler, device, barrier)
     res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier, fp8=fp8)
     if res["status"] != 0:
         raise SystemExit(f"device status {res['status']} after the timed region")
@@ -555,7 +563,8 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
-            "config": _config(w, res["sets"], res["resident_mb"]),
+            "config": _config(w, res["sets"], res["resident_mb"], "replicas (one independent step per GPU)"
+                              if ws > 1 else "one GPU"),
             ("pct_of_e4m3_peak" if fp8 else "pct_of_bf16_peak"): 100.0 * (value / ws) / peak,
             "roofline": roof, "clocks": sampler.summary(), "gpu_launches": res["launches"]}
     if res["merge_ms"]:
@@ -585,27 +594,201 @@ def run_ours(args):
     return 0
 
 
-def fused_timing(pa, w, steps, warmup, device):
-    """Device time of one pa_attn_fwd_chunks launch over the workload's chunks."""
+def shard_sizes(n: int, world: int):
+    """Sequence shard lengths of n rows over `world` ranks (the first n %
+    world ranks take one row more)."""
+    return [n // world + (1 if r < n % world else 0) for r in range(world)]
+
+
+def run_ring(args, pa, w, peaks, sampler, device, barrier):
+    """Ring Attention over the process group: rank r holds shard r of the
+    query rows and of the K/V rows of workload `w` and runs
+    context_parallel.ring_attention.  Value = the whole problem's FLOPs per
+    step over the slowest rank's time (strong scaling)."""
+    import dataclasses
+
     import torch
-    q, k, v = workloads.make_case(w, device=device)
-    pairs = workloads.split_keys(k, v, w.chunks)
-    del k, v
-    kc, vc = [a for a, _ in pairs], [b for _, b in pairs]
-    o = torch.empty_like(q)
-    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
-    for _ in range(warmup):
-        pa.attn_fwd_chunks(q, kc, vc, scale=w.scale, out=o, lse=lse)
+    import torch.distributed as dist
+    from context_blocks_b200 import context_parallel as cp
+
+    ws, rank = dist.get_world_size(), dist.get_rank()
+    nq_all, nk_all = shard_sizes(w.Nq, ws), shard_sizes(w.Nk, ws)
+    wr = dataclasses.replace(w, Nq=nq_all[rank], Nk=nk_all[rank], chunks=(nk_all[rank],), seed=w.seed + 100 * rank)
+    q, k, v = workloads.make_case(wr, device=device)
+    out = torch.empty_like(q)
+    comm = torch.cuda.Stream(device=device)
+    fwd_ev = ([], [])
+
+    def attend_timed(qq, kk, vv, o_acc, lse_acc, first, final, o, scale):
+        fwd_ev[0].append(_record())
+        pa.attn_fwd_accum(qq, kk, vv, o_acc, lse_acc, first=first, final=final, out=o, scale=scale)
+        fwd_ev[1].append(_record())
+
+    def step(timed=False):
+        return cp.ring_attention(q, k, v, kv_lens=nk_all, scale=w.scale, out=out, comm_stream=comm,
+                                 attend=attend_timed if timed else None)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
-        pa.attn_fwd_chunks(q, kc, vc, scale=w.scale, out=o, lse=lse)
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
+    with sampler:
+        t0.record()
+        for _ in range(args.steps):
+            step(timed=True)
+        t1.record()
+        torch.cuda.synchronize()
+    barrier()
+    status = pa.poll_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed region")
+    max_ms = max_over_ranks(t0.elapsed_time(t1), device)
     fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
-    return {"step_ms": ms, "tflops_step": fl / (ms * 1e-3) / 1e12, "launches_per_step": 1}
+    value = fl * args.steps / (max_ms * 1e-3) / 1e12
+    fwd_ms = [a.elapsed_time(b) for a, b in zip(*fwd_ev)]
+    # the fold kernel: this rank's FLOPs per ring pass over its launches
+    fl_rank = workloads.flops(w.B, w.H, nq_all[rank], w.Nk, w.d)
+    launch_ms = statistics.fmean(fwd_ms)
+    achieved = fl_rank / ws / (launch_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": None, "kernel": f"attn_fwd_kernel<{w.d}, false> (accumulate mode)", "launch_ms": launch_ms,
+            "peak_basis": f"{peaks['source']} burst bf16 (MEASURED_PEAKS.json bf16_tflops), rank {rank}"}
+    # End to end: each step uploads this rank's shards from pinned host
+    # memory, runs the ring, downloads this rank's output and LSE.
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hl = torch.empty(out.shape[:3], dtype=torch.float32, pin_memory=True)
+    e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        o, lse = step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(_config(w, parallelism=f"ring attention over {ws} ranks (NCCL P2P on a second stream)"),
+                           q_shards=nq_all, kv_shards=nk_all,
+                           l2="each rank's K/V blocks rotate through the ring; inputs far larger than L2"),
+            "pct_of_bf16_peak": 100.0 * (value / ws) / peak, "roofline": roof, "clocks": sampler.summary(),
+            "gpu_launches": args.steps * ws,
+            "e2e": {"value": fl * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
+                    "d2h_bytes_per_step": int(out.numel() * 2 + out.numel() // w.d * 4), "steps": e_steps,
+                    "note": "per rank; every rank moves its own shards"}}
+    barrier()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+    return 0
+
+
+class ModeSets:
+    """Rotating input sets for one way of running a chunked workload:
+    ``chunks`` = pa_attn_fwd per chunk, then pa_attn_merge; ``fused`` = one
+    pa_attn_fwd_chunks launch; ``fold`` = pa_attn_fwd_accum per chunk into an
+    fp32 running state, the last fold writing the bf16 output.  Enough sets
+    that consecutive steps read inputs totalling more than L2."""
+
+    def __init__(self, pa, w, mode, device):
+        import torch
+        self.pa, self.w, self.mode = pa, w, mode
+        self.sets = []
+        n = len(w.chunks)
+        for s in range(_sets_for(w)):
+            q, k, v = workloads.make_case(w, device=device, seed=w.seed + 1000 * s)
+            pairs = workloads.split_keys(k, v, w.chunks)
+            del k, v
+            st = {"q": q, "k": [a for a, _ in pairs], "v": [b for _, b in pairs], "o": torch.empty_like(q),
+                  "lse": torch.empty(q.shape[:3], dtype=torch.float32, device=device)}
+            if mode == "chunks" and n > 1:
+                st["o_parts"] = torch.empty((n,) + tuple(q.shape), dtype=torch.bfloat16, device=device)
+                st["lse_parts"] = torch.empty((n,) + tuple(q.shape[:3]), dtype=torch.float32, device=device)
+            if mode == "fold":
+                st["o_acc"] = torch.empty(q.shape, dtype=torch.float32, device=device)
+            self.sets.append(st)
+        self.launches = {"chunks": n + (1 if n > 1 else 0), "fused": 1, "fold": n}[mode]
+
+    def run(self, i):
+        pa, w, st = self.pa, self.w, self.sets[i % len(self.sets)]
+        if self.mode == "chunks":
+            pa.blockwise_attention(st["q"], st["k"], st["v"], scale=w.scale, o_parts=st.get("o_parts"),
+                                   lse_parts=st.get("lse_parts"), out=st["o"], lse=st["lse"])
+        elif self.mode == "fused":
+            pa.attn_fwd_chunks(st["q"], st["k"], st["v"], scale=w.scale, out=st["o"], lse=st["lse"])
+        else:
+            n = len(st["k"])
+            for c in range(n):
+                pa.attn_fwd_accum(st["q"], st["k"][c], st["v"][c], st["o_acc"], st["lse"], first=(c == 0),
+                                  final=(c == n - 1), out=st["o"] if c == n - 1 else None, scale=w.scale)
+
+
+def mode_timing(pa, w, mode, steps, warmup, device, graph=False):
+    """Device time per step of `mode` on workload `w` (CUDA events on the
+    launching stream).  With ``graph`` the steps are captured once in a CUDA
+    graph (one pass over the rotating sets) and replayed, so the host-side
+    cost of each library call (argument checks, tensor-map encoding, Python)
+    drops out and what remains is the GPU's own time."""
+    import torch
+    ms_sets = ModeSets(pa, w, mode, device)
+    nsets = len(ms_sets.sets)
+    side = torch.cuda.Stream(device=device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(side):
+        for i in range(max(warmup, nsets)):
+            ms_sets.run(i)
+    torch.cuda.current_stream(device).wait_stream(side)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for i in range(nsets):
+                ms_sets.run(i)
+        g.replay()
+        torch.cuda.synchronize()
+        reps = max(1, steps // nsets)
+        t0.record()
+        for _ in range(reps):
+            g.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        n_steps = reps * nsets
+        del g
+    else:
+        t0.record()
+        for i in range(steps):
+            ms_sets.run(i)
+        t1.record()
+        torch.cuda.synchronize()
+        n_steps = steps
+    ms = t0.elapsed_time(t1) / n_steps
+    status = pa.poll_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after timing {w.name} {mode}")
+    del ms_sets
+    torch.cuda.empty_cache()
+    fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
+    return {"step_ms": ms, "tflops_step": fl / (ms * 1e-3) / 1e12, "launches_per_step":
+            {"chunks": len(w.chunks) + (1 if len(w.chunks) > 1 else 0), "fused": 1, "fold": len(w.chunks)}[mode],
+            "timing": "CUDA graph replay" if graph else "eager launches"}
 
 
 def fp8_timing(pa, w, steps, warmup, device):
@@ -638,26 +821,37 @@ def extra_measurements(pa, device, peaks):
     """Secondary lines: the other workloads' device throughput (not the
     headline value).  Bounded repetitions each."""
     out = {}
-    plan = [("ring", 20, 3), ("tails", 10, 3), ("flux1008", 10, 3), ("hunyuan", 3, 1)]
-    for name, steps, warm in plan:
+    # The FLUX.1-dev 1024^2 shape, per launch, as the headline is timed.
+    wf = workloads.get("flux")
+    r = time_workload(pa, wf, 200, 10, device)
+    fl = workloads.flops(wf.B, wf.H, wf.Nq, wf.Nk, wf.d)
+    out["flux"] = {"step_ms": r["total_ms"] / 200, "fwd_ms_per_launch": statistics.fmean(r["fwd_ms"]),
+                   "fwd_tflops": fl / (statistics.fmean(r["fwd_ms"]) * 1e-3) / 1e12}
+    out["flux"]["frac_of_bf16_peak"] = out["flux"]["fwd_tflops"] / peaks["bf16_tflops"]
+    # Chunked workloads: per-chunk forward + merge with per-launch events
+    # (eager), then every mode timed from CUDA-graph replays (device time).
+    for name, steps in (("ring", 20), ("tails", 10), ("flux1008", 10)):
         w = workloads.get(name)
-        r = time_workload(pa, w, steps, warm, device)
+        r = time_workload(pa, w, steps, 3, device)
         fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
         ent = {"step_ms": r["total_ms"] / steps, "tflops_step": fl * steps / (r["total_ms"] * 1e-3) / 1e12,
                "fwd_ms_per_launch": statistics.fmean(r["fwd_ms"]),
-               "fwd_tflops": (fl / len(w.chunks)) / (statistics.fmean(r["fwd_ms"]) * 1e-3) / 1e12}
+               "fwd_tflops": (fl / len(w.chunks)) / (statistics.fmean(r["fwd_ms"]) * 1e-3) / 1e12,
+               "timing": "eager launches, events around each launch"}
         if r["merge_ms"]:
             mb = workloads.merge_bytes(len(w.chunks), w.B, w.H, w.Nq, w.d)
             ent["merge_ms"] = statistics.fmean(r["merge_ms"])
             ent["merge_gbs"] = mb / (ent["merge_ms"] * 1e-3) / 1e9
         ent["pct_of_bf16_peak"] = 100.0 * ent["fwd_tflops"] / peaks["bf16_tflops"]
         out[name] = ent
-    # The chunked workloads as one fused launch (pa_attn_fwd_chunks).
-    for name in ("ring", "tails", "flux1008"):
-        w = workloads.get(name)
-        out[name + "_fused"] = fused_timing(pa, w, steps=20, warmup=3, device=device)
-    out["hunyuan_8chunks_fused"] = fused_timing(
-        pa, workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8), steps=2, warmup=1, device=device)
+        for mode in ("chunks", "fused", "fold"):
+            g = mode_timing(pa, w, mode, 200, 3, device, graph=True)
+            g["frac_of_bf16_peak"] = g["tflops_step"] / peaks["bf16_tflops"]
+            out[f"{name}_{mode}_graph"] = g
+        out[name + "_fused"] = mode_timing(pa, w, "fused", 20, 3, device)
+    w8 = workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8)
+    for mode in ("fused", "fold"):
+        out[f"hunyuan_8chunks_{mode}"] = mode_timing(pa, w8, mode, 2, 1, device)
     # The e4m3 forward on the FLUX and HunyuanVideo shapes; its peak is the
     # measured bf16 burst figure times the nominal fp8/bf16 ratio of 2.
     for name, steps in (("flux", 20), ("hunyuan", 2)):
@@ -687,12 +881,6 @@ def extra_measurements(pa, device, peaks):
                             "gbs": 3.0 * x.numel() / (ms * 1e-3) / 1e9,
                             "frac_of_hbm": 3.0 * x.numel() / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     del x, q8
-    # The CTA-pair forward kernel (pa_attn_fwd_pair) on the FLUX-shaped workload.
-    wf = workloads.get("flux")
-    r = time_workload(pa, wf, 200, 10, device, pair=True)
-    fl = workloads.flops(wf.B, wf.H, wf.Nq, wf.Nk, wf.d)
-    out["flux_pair_kernel"] = {"fwd_ms_per_launch": statistics.fmean(r["fwd_ms"]),
-                               "fwd_tflops": fl / (statistics.fmean(r["fwd_ms"]) * 1e-3) / 1e12}
     w8 = workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8)
     r = time_workload(pa, w8, 2, 1, device)
     fl = workloads.flops(w8.B, w8.H, w8.Nq, w8.Nk, w8.d)
@@ -708,10 +896,12 @@ def extra_measurements(pa, device, peaks):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="flux", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="hunyuan", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--parallel", choices=["ring", "replicas"], default="ring",
+                    help="with more than one GPU: ring attention over the ranks, or independent replicas")
     ap.add_argument("--fp8", action="store_true",
                     help="time the e4m3 forward (pa_attn_fwd_fp8) instead of bf16; one-chunk workloads")
     ap.add_argument("--heads", type=int, default=None,
