@@ -11,7 +11,9 @@
 // real length never enter the softmax (section "Ring Anything Attention":
 // blocks are trimmed back to their real length before attention).
 //
-// Kernel structure (one CTA per 256 query rows of one (b, h)):
+// Kernel structure (persistent: each CTA walks work items, an item being 256
+// query rows of one (b, h); the next item's Q load and first Q K^T overlap the
+// current item's last tiles and epilogue):
 //   warps 0-3  softmax warpgroup for query tile 0 (rows   0..127 of the block)
 //   warps 4-7  softmax warpgroup for query tile 1 (rows 128..255 of the block)
 //   warp  8    TMEM allocation + tcgen05.mma issue (the whole warp runs the
@@ -94,8 +96,8 @@ struct FwdLayout {
   static constexpr int kRingOff = kQOff + kQTiles * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
   // q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain,
-  // p_part[2][3] (parts of P before the last, which arrives on p_full)
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 6;
+  // p_part[2][3] (parts of P before the last, which arrives on p_full), q_empty
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 6 + 1;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
   static constexpr int kBytes = kAbortOff + 4;
@@ -130,13 +132,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t bar_o_full0 = bars + 8 * (6 + 2 * kStages);
   const uint32_t bar_drain = bars + 8 * (8 + 2 * kStages);
   const uint32_t bar_p_part0 = bars + 8 * (9 + 2 * kStages);  // + 8 * (3 * i + part)
+  const uint32_t bar_q_empty = bars + 8 * (15 + 2 * kStages);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kTmemSlotOff);
   volatile int* abort_word = reinterpret_cast<volatile int*>(gbase + L::kAbortOff);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int q0 = blockIdx.x * (kQTiles * kBM);
-  const int bh = blockIdx.y;
   const int n = p.n_kv_tiles;
   const uint64_t lim = p.timeout_ns;
 
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar_o_full0 + 8 * i, 1);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_q_empty, 1);
     *abort_word = 0;
     fence_barrier_init();
   }
@@ -176,49 +178,62 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ------------------------------------------------------------ producer
     // The whole warp runs the loop in step; the elected lane issues the loads.
     const bool leader = elect_one();
-    if (leader) {
-      for (int i = 0; i < kQTiles; ++i) {
-        mbar_arrive_expect_tx(bar_q_full0 + 8 * i, L::kTileBytes);
-#pragma unroll
-        for (int b = 0; b < L::kBoxes; ++b)
-          tma_load_3d(sQ + i * L::kTileBytes + b * L::kBoxBytes, &tm_q, bar_q_full0 + 8 * i, b * L::kBoxCols,
-                      q0 + i * kBM, bh);
-      }
-    }
-    __syncwarp();
     bool ok = true;
-    int idx = 0;  // ring loads issued so far
-    for (int jt = 0; jt < n && ok; ++jt) {
-      // Chunk of key tile jt and the tile's row offset inside that chunk.
-      int c = 0;
-#pragma unroll
-      for (int cc = 1; cc < kMaxChunks; ++cc) c += (jt >= kv.tile_start[cc]) ? 1 : 0;
-      const int row0 = (jt - kv.tile_start[c]) * kBN;
-      for (int t = 0; t < 2; ++t) {  // t = 0: K tile, t = 1: V tile
-        const int s = idx % kStages;
-        const uint32_t u = idx / kStages;
-        const bool got = mbar_wait(bar_kv_empty0 + 8 * s, (u & 1) ^ 1, abort_word, p.status, kStatusTimeout, lim);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        if (leader) {
-          const uint32_t full = bar_kv_full0 + 8 * s;
-          mbar_arrive_expect_tx(full, L::kTileBytes);
-          const CUtensorMap* map = t ? &kv.v[c] : &kv.k[c];
+    int idx = 0;      // ring loads issued so far (over all items)
+    int q_loads = 0;  // items whose Q was issued
+    for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
+      const int bh = item / p.blocks_per_bh;
+      const int q0 = (item % p.blocks_per_bh) * (kQTiles * kBM);
+      // Q of this item once every Q K^T of the previous one has completed.
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_q_empty, (q_loads & 1) ^ 1, abort_word, p.status, kStatusTimeout,
+                                             lim))) {
+        ok = false;
+        break;
+      }
+      if (leader) {
+        for (int i = 0; i < kQTiles; ++i) {
+          mbar_arrive_expect_tx(bar_q_full0 + 8 * i, L::kTileBytes);
 #pragma unroll
           for (int b = 0; b < L::kBoxes; ++b)
-            tma_load_3d(sRing + s * L::kTileBytes + b * L::kBoxBytes, map, full, b * L::kBoxCols, row0, bh);
+            tma_load_3d(sQ + i * L::kTileBytes + b * L::kBoxBytes, &tm_q, bar_q_full0 + 8 * i, b * L::kBoxCols,
+                        q0 + i * kBM, bh);
         }
-        __syncwarp();
-        ++idx;
+      }
+      __syncwarp();
+      ++q_loads;
+      for (int jt = 0; jt < n && ok; ++jt) {
+        // Chunk of key tile jt and the tile's row offset inside that chunk.
+        int c = 0;
+#pragma unroll
+        for (int cc = 1; cc < kMaxChunks; ++cc) c += (jt >= kv.tile_start[cc]) ? 1 : 0;
+        const int row0 = (jt - kv.tile_start[c]) * kBN;
+        for (int t = 0; t < 2; ++t) {  // t = 0: K tile, t = 1: V tile
+          const int s = idx % kStages;
+          const uint32_t u = idx / kStages;
+          const bool got = mbar_wait(bar_kv_empty0 + 8 * s, (u & 1) ^ 1, abort_word, p.status, kStatusTimeout, lim);
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+          if (leader) {
+            const uint32_t full = bar_kv_full0 + 8 * s;
+            mbar_arrive_expect_tx(full, L::kTileBytes);
+            const CUtensorMap* map = t ? &kv.v[c] : &kv.k[c];
+#pragma unroll
+            for (int b = 0; b < L::kBoxes; ++b)
+              tma_load_3d(sRing + s * L::kTileBytes + b * L::kBoxBytes, map, full, b * L::kBoxCols, row0, bh);
+          }
+          __syncwarp();
+          ++idx;
+        }
       }
     }
     if (!ok) {
       // Aborted: let every copy already in flight land before the CTA exits.
       // Slot s received ceil((idx - s) / kStages) loads; wait for the last.
-      for (int i = 0; i < kQTiles; ++i)
-        mbar_wait(bar_q_full0 + 8 * i, 0, nullptr, p.status, kStatusTimeout, lim);
+      if (q_loads > 0)
+        for (int i = 0; i < kQTiles; ++i)
+          mbar_wait(bar_q_full0 + 8 * i, (q_loads - 1) & 1, nullptr, p.status, kStatusTimeout, lim);
       for (int s = 0; s < kStages && s < idx; ++s) {
         const int cnt = (idx - s + kStages - 1) / kStages;
         mbar_wait(bar_kv_full0 + 8 * s, (cnt - 1) & 1, nullptr, p.status, kStatusTimeout, lim);
@@ -277,72 +292,84 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // P.V accumulates.
     const bool o_loaded = (p.acc_o != nullptr) && !(p.acc_flags & kAccFirst);
 
-    bool ok = wait_all(bar_q_full0, 0) && wait_all(bar_q_full0 + 8, 0) && wait_all(bar_kv_full0, 0);
-    if (ok) {
-      tc_fence_after();
-      if (leader) {
-        issue_qk(0, 0);
-        umma_commit(bar_s_full0);
-        issue_qk(1, 0);
-        umma_commit(bar_s_full0 + 8);
-        umma_commit(bar_kv_empty0);
-      }
-      __syncwarp();
-    }
-    int idx = 1;
-    for (int j = 0; j < n && ok; ++j) {
-      const int sv = idx % kStages;
-      const uint32_t uv = idx / kStages;
-      ++idx;
-      int sk = 0;
-      uint32_t uk = 0;
-      const bool more = (j + 1 < n);
-      if (more) {
-        sk = idx % kStages;
-        uk = idx / kStages;
-        ++idx;
-      }
-      if (!wait_all(bar_kv_full0 + 8 * sv, uv & 1)) {
+    bool ok = true;
+    int idx = 0;  // ring position (over all items)
+    int g = 0;    // key tiles over all items: phases of the S and P barriers
+    int t = 0;    // items of this CTA
+    for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++t) {
+      if (!wait_all(bar_q_full0, t & 1) || !wait_all(bar_q_full0 + 8, t & 1) ||
+          !wait_all(bar_kv_full0 + 8 * (idx % kStages), (idx / kStages) & 1)) {
         ok = false;
         break;
       }
-      for (int i = 0; i < 2; ++i) {
-        // P.V part by part: part q covers keys [q, q + 1) * kBN / kPParts.
-        constexpr int kKkPerPart = (kBN / kKPerMma) / kPParts;
-        for (int q = 0; q < kPParts - 1 && ok; ++q) {
-          if (!wait_all(bar_p_part0 + 8 * (3 * i + q), j & 1)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (leader) issue_pv(i, sv, o_loaded || j > 0 || q > 0, q * kKkPerPart, (q + 1) * kKkPerPart);
-          __syncwarp();
+      tc_fence_after();
+      if (leader) {
+        issue_qk(0, idx % kStages);
+        umma_commit(bar_s_full0);
+        issue_qk(1, idx % kStages);
+        umma_commit(bar_s_full0 + 8);
+        umma_commit(bar_kv_empty0 + 8 * (idx % kStages));
+        if (n == 1) umma_commit(bar_q_empty);
+      }
+      __syncwarp();
+      ++idx;
+      for (int j = 0; j < n && ok; ++j, ++g) {
+        const int sv = idx % kStages;
+        const uint32_t uv = idx / kStages;
+        ++idx;
+        int sk = 0;
+        uint32_t uk = 0;
+        const bool more = (j + 1 < n);
+        if (more) {
+          sk = idx % kStages;
+          uk = idx / kStages;
+          ++idx;
         }
-        if (!ok || !wait_all(bar_p_full0 + 8 * i, j & 1)) {
+        if (!wait_all(bar_kv_full0 + 8 * sv, uv & 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (leader) issue_pv(i, sv, true, (kPParts - 1) * kKkPerPart, kBN / kKPerMma);
-        if (leader && i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
-        __syncwarp();
-        if (more) {
-          if (i == 0) {
-            if (!wait_all(bar_kv_full0 + 8 * sk, uk & 1)) {
+        for (int i = 0; i < 2; ++i) {
+          // P.V part by part: part q covers keys [q, q + 1) * kBN / kPParts.
+          constexpr int kKkPerPart = (kBN / kKPerMma) / kPParts;
+          for (int q = 0; q < kPParts - 1 && ok; ++q) {
+            if (!wait_all(bar_p_part0 + 8 * (3 * i + q), g & 1)) {
               ok = false;
               break;
             }
             tc_fence_after();
+            if (leader) issue_pv(i, sv, o_loaded || j > 0 || q > 0, q * kKkPerPart, (q + 1) * kKkPerPart);
+            __syncwarp();
           }
-          if (leader) {
-            issue_qk(i, sk);
-            umma_commit(bar_s_full0 + 8 * i);
-            if (i == 1) umma_commit(bar_kv_empty0 + 8 * sk);
+          if (!ok || !wait_all(bar_p_full0 + 8 * i, g & 1)) {
+            ok = false;
+            break;
           }
-        } else if (leader) {
-          umma_commit(bar_o_full0 + 8 * i);
+          tc_fence_after();
+          if (leader) issue_pv(i, sv, true, (kPParts - 1) * kKkPerPart, kBN / kKPerMma);
+          if (leader && i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
+          __syncwarp();
+          if (more) {
+            if (i == 0) {
+              if (!wait_all(bar_kv_full0 + 8 * sk, uk & 1)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            if (leader) {
+              issue_qk(i, sk);
+              umma_commit(bar_s_full0 + 8 * i);
+              if (i == 1) {
+                umma_commit(bar_kv_empty0 + 8 * sk);
+                if (j + 2 == n) umma_commit(bar_q_empty);  // the item's last Q K^T
+              }
+            }
+          } else if (leader) {
+            umma_commit(bar_o_full0 + 8 * i);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
     // Every MMA issued completes before tensor memory is freed.
@@ -357,9 +384,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + i * kBN + lane_off;
     const uint32_t tO = tmem + 2 * kBN + i * D + lane_off;
-    const int row = q0 + i * kBM + t;
-    const bool in_range = row < p.Nq;
-    const size_t row_idx = static_cast<size_t>(bh) * p.Nq + row;
     // Logit scale in log2 units; e4m3 inputs may carry their dequantisation
     // scales in device memory, which are checked here: a scale that is not
     // finite and positive is reported in the status word (the outputs are then
@@ -378,192 +402,209 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         o_mul = p.o_scale;
       }
     }
-    float m_ref = -INFINITY;
-    float l = 0.f;
-    bool ok = true;
-    // Accumulate mode: start from the caller's running (O, LSE) instead of an
-    // empty state.  Rows past Nq and rows whose running LSE is -inf (no key
-    // seen yet) start empty, with O = 0.
     const bool o_loaded = (p.acc_o != nullptr) && !(p.acc_flags & kAccFirst);
-    if (o_loaded) {
-      const float lse0 = in_range ? p.acc_lse[row_idx] : -INFINITY;
-      const bool have = lse0 > -INFINITY;
-      if (have) {
-        m_ref = lse0 * 1.4426950408889634f;
-        l = 1.f;
-      }
-      const float4* src = reinterpret_cast<const float4*>(p.acc_o + row_idx * D);
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t orr[32];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const float4 x = have ? __ldg(src + ch * 8 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-          orr[4 * v] = __float_as_uint(x.x);
-          orr[4 * v + 1] = __float_as_uint(x.y);
-          orr[4 * v + 2] = __float_as_uint(x.z);
-          orr[4 * v + 3] = __float_as_uint(x.w);
+    bool ok = true;
+    int g = 0;   // key tiles over all items: phases of the S barrier
+    int it = 0;  // items of this CTA: phase of the O barrier
+    // This thread's query row of an item, and its index in [B*H, Nq]
+    // (recomputed where needed rather than kept live through the key loop).
+    auto row_of = [&](int item) { return (item % p.blocks_per_bh) * (kQTiles * kBM) + i * kBM + t; };
+    auto index_of = [&](int item) {
+      return static_cast<size_t>(item / p.blocks_per_bh) * p.Nq + row_of(item);
+    };
+    for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x, ++it) {
+      float m_ref = -INFINITY;
+      float l = 0.f;
+      // Accumulate mode: start from the caller's running (O, LSE) instead of
+      // an empty state.  Rows past Nq and rows whose running LSE is -inf (no
+      // key seen yet) start empty, with O = 0.  (This warpgroup's epilogue of
+      // the previous item has read O out; its P V are complete.)
+      if (o_loaded) {
+        const bool in_range = row_of(item) < p.Nq;
+        const size_t row_idx = index_of(item);
+        const float lse0 = in_range ? p.acc_lse[row_idx] : -INFINITY;
+        const bool have = lse0 > -INFINITY;
+        if (have) {
+          m_ref = lse0 * 1.4426950408889634f;
+          l = 1.f;
         }
-        tmem_st_x32(tO + ch * 32, orr);
-      }
-      tmem_st_wait();
-    }
-
-    for (int j = 0; j < n; ++j) {
-      // Chunk of key tile j, from the prefix tile counts (no state carried).
-      int chunk = 0;
-#pragma unroll
-      for (int cc = 1; cc < kMaxChunks; ++cc) chunk += (j >= kv.tile_start[cc]) ? 1 : 0;
-      const int valid = kv.nk[chunk] - (j - kv.tile_start[chunk]) * kBN;  // keys of this tile in its chunk
-      const bool got =
-          mbar_wait_hint(bar_s_full0 + 8 * i, j & 1, abort_word, p.status, kStatusTimeout, lim, kSuspendHintNs);
-      if (__any_sync(0xffffffffu, !got)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sr[kBN];
-      tmem_ld_x128(tS, sr);
-      float s[kBN];
-#pragma unroll
-      for (int e = 0; e < kBN; ++e) s[e] = __uint_as_float(sr[e]);
-      if (valid < kBN) {
-#pragma unroll
-        for (int e = 0; e < kBN; ++e)
-          if (e >= valid) s[e] = -INFINITY;
-      }
-      // Row max: 8 independent chains of 3-input max.
-      float m8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
-#pragma unroll
-      for (int e = 16; e < kBN; e += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = max3f(m8[k], s[e + k], s[e + 8 + k]);
-      float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], max3f(m8[5], m8[6], m8[7])));
-      mx *= c;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mx > m_ref + kRescaleLog2) {
-        alpha = ex2_approx(m_ref - mx);  // 0 when the row was empty (m_ref = -inf)
-        l *= alpha;
-        m_ref = mx;
-        rescale = (j > 0) || o_loaded;
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
-        // PV of tile j-1 has completed: S_i(j) was issued after it and the
-        // tcgen05 ops of the issuing thread complete in order.  (On tile 0 of
-        // a fold, O holds the loaded state this thread stored.)
+        const float4* src = reinterpret_cast<const float4*>(p.acc_o + row_idx * D);
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t orr[32];
-          tmem_ld_x32(tO + ch * 32, orr);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+          for (int v = 0; v < 8; ++v) {
+            const float4 x = have ? __ldg(src + ch * 8 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+            orr[4 * v] = __float_as_uint(x.x);
+            orr[4 * v + 1] = __float_as_uint(x.y);
+            orr[4 * v + 2] = __float_as_uint(x.z);
+            orr[4 * v + 3] = __float_as_uint(x.w);
+          }
           tmem_st_x32(tO + ch * 32, orr);
         }
+        tmem_st_wait();
       }
-      // x = s * c - m_ref on packed pairs, P = 2^x on MUFU, the row sum in
-      // four packed partial sums.
-      const float neg_m = -m_ref;
-      const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
-      uint64_t l4[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-#pragma unroll
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float x0, x1;
-          f2_split(f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2), x0, x1);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          l4[e & 3] = f2_add(l4[e & 3], f2(p0, p1));
-          if constexpr (kFp8) {
-            // four e4m3 keys per 32-bit column, lowest key in the low byte
-            const uint32_t h = pack_e4m3x2(p0, p1);
-            if (e & 1)
-              pk[e >> 1] |= h << 16;
-            else
-              pk[e >> 1] = h;
-          } else {
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-        }
-        if constexpr (kFp8) {
-          const uint32_t(&pk8)[8] = *reinterpret_cast<const uint32_t(*)[8]>(pk);
-          tmem_st_x8(tS + ch * 8, pk8);
-        } else {
-          tmem_st_x16(tS + ch * 16, pk);
-        }
-        constexpr int kChPerPart = (kBN / 32) / kPParts;  // 32-key chunks per part
-        if ((ch + 1) % kChPerPart == 0 && ch + 1 < kBN / 32) {
-          // Part (ch + 1) / kChPerPart - 1 of P is in TMEM: hand it over.
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_p_part0 + 8 * (3 * i + (ch + 1) / kChPerPart - 1));
-        }
-      }
-      {
-        const uint64_t sum = f2_add(f2_add(l4[0], l4[1]), f2_add(l4[2], l4[3]));
-        float a, b;
-        f2_split(sum, a, b);
-        l += a + b;
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p_full0 + 8 * i);
-    }
 
-    if (ok) {
-      const bool got = mbar_wait(bar_o_full0 + 8 * i, 0, abort_word, p.status, kStatusTimeout, lim);
-      ok = !__any_sync(0xffffffffu, !got);
-    }
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = o_mul / l;
-      const float lse_out = (m_ref + lg2_approx(l)) * 0.69314718055994531f;
-      const bool state_out = (p.acc_o != nullptr) && !(p.acc_flags & kAccFinal);
-      if (state_out) {
-        // Running state: normalised fp32 O and its LSE.
-        float4* dst = reinterpret_cast<float4*>(p.acc_o + row_idx * D);
+      for (int j = 0; j < n; ++j, ++g) {
+        // Chunk of key tile j, from the prefix tile counts (no state carried).
+        int chunk = 0;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t orr[32];
-          tmem_ld_x32(tO + ch * 32, orr);
-          if (in_range) {
+        for (int cc = 1; cc < kMaxChunks; ++cc) chunk += (j >= kv.tile_start[cc]) ? 1 : 0;
+        const int valid = kv.nk[chunk] - (j - kv.tile_start[chunk]) * kBN;  // keys of this tile in its chunk
+        const bool got =
+            mbar_wait_hint(bar_s_full0 + 8 * i, g & 1, abort_word, p.status, kStatusTimeout, lim, kSuspendHintNs);
+        if (__any_sync(0xffffffffu, !got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[kBN];
+        tmem_ld_x128(tS, sr);
+        float s[kBN];
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[ch * 8 + v] = make_float4(__uint_as_float(orr[4 * v]) * inv_l, __uint_as_float(orr[4 * v + 1]) * inv_l,
-                                            __uint_as_float(orr[4 * v + 2]) * inv_l,
-                                            __uint_as_float(orr[4 * v + 3]) * inv_l);
+        for (int e = 0; e < kBN; ++e) s[e] = __uint_as_float(sr[e]);
+        if (valid < kBN) {
+#pragma unroll
+          for (int e = 0; e < kBN; ++e)
+            if (e >= valid) s[e] = -INFINITY;
+        }
+        // Row max: 8 independent chains of 3-input max.
+        float m8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+        for (int e = 16; e < kBN; e += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = max3f(m8[k], s[e + k], s[e + 8 + k]);
+        float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], max3f(m8[5], m8[6], m8[7])));
+        mx *= c;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mx > m_ref + kRescaleLog2) {
+          alpha = ex2_approx(m_ref - mx);  // 0 when the row was empty (m_ref = -inf)
+          l *= alpha;
+          m_ref = mx;
+          rescale = (j > 0) || o_loaded;
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+          // PV of tile j-1 has completed: S_i(j) was issued after it and the
+          // tcgen05 ops of the issuing thread complete in order.  (On tile 0 of
+          // a fold, O holds the loaded state this thread stored.)
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t orr[32];
+            tmem_ld_x32(tO + ch * 32, orr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st_x32(tO + ch * 32, orr);
           }
         }
-      } else {
-        __nv_bfloat16* orow = p.o + row_idx * D;
+        // x = s * c - m_ref on packed pairs, P = 2^x on MUFU, the row sum in
+        // four packed partial sums.
+        const float neg_m = -m_ref;
+        const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
+        uint64_t l4[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t orr[32];
-          tmem_ld_x32(tO + ch * 32, orr);
+        for (int ch = 0; ch < kBN / 32; ++ch) {
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
-          if (in_range) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int e = 0; e < 16; ++e) {
+            float x0, x1;
+            f2_split(f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2), x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            l4[e & 3] = f2_add(l4[e & 3], f2(p0, p1));
+            if constexpr (kFp8) {
+              // four e4m3 keys per 32-bit column, lowest key in the low byte
+              const uint32_t h = pack_e4m3x2(p0, p1);
+              if (e & 1)
+                pk[e >> 1] |= h << 16;
+              else
+                pk[e >> 1] = h;
+            } else {
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+          }
+          if constexpr (kFp8) {
+            const uint32_t(&pk8)[8] = *reinterpret_cast<const uint32_t(*)[8]>(pk);
+            tmem_st_x8(tS + ch * 8, pk8);
+          } else {
+            tmem_st_x16(tS + ch * 16, pk);
+          }
+          constexpr int kChPerPart = (kBN / 32) / kPParts;  // 32-key chunks per part
+          if ((ch + 1) % kChPerPart == 0 && ch + 1 < kBN / 32) {
+            // Part (ch + 1) / kChPerPart - 1 of P is in TMEM: hand it over.
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p_part0 + 8 * (3 * i + (ch + 1) / kChPerPart - 1));
           }
         }
+        {
+          const uint64_t sum = f2_add(f2_add(l4[0], l4[1]), f2_add(l4[2], l4[3]));
+          float a, b;
+          f2_split(sum, a, b);
+          l += a + b;
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p_full0 + 8 * i);
       }
-      if (in_range) {
-        if (p.acc_o != nullptr)
-          p.acc_lse[row_idx] = lse_out;
-        else
-          p.lse[row_idx] = lse_out;
+
+      if (!ok) break;
+      {
+        const bool got = mbar_wait(bar_o_full0 + 8 * i, it & 1, abort_word, p.status, kStatusTimeout, lim);
+        ok = !__any_sync(0xffffffffu, !got);
       }
+      if (ok) {
+        tc_fence_after();
+        const bool in_range = row_of(item) < p.Nq;
+        const size_t row_idx = index_of(item);
+        const float inv_l = o_mul / l;
+        const float lse_out = (m_ref + lg2_approx(l)) * 0.69314718055994531f;
+        const bool state_out = (p.acc_o != nullptr) && !(p.acc_flags & kAccFinal);
+        if (state_out) {
+          // Running state: normalised fp32 O and its LSE.
+          float4* dst = reinterpret_cast<float4*>(p.acc_o + row_idx * D);
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t orr[32];
+            tmem_ld_x32(tO + ch * 32, orr);
+            if (in_range) {
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[ch * 8 + v] = make_float4(__uint_as_float(orr[4 * v]) * inv_l, __uint_as_float(orr[4 * v + 1]) * inv_l,
+                                              __uint_as_float(orr[4 * v + 2]) * inv_l,
+                                              __uint_as_float(orr[4 * v + 3]) * inv_l);
+            }
+          }
+        } else {
+          __nv_bfloat16* orow = p.o + row_idx * D;
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t orr[32];
+            tmem_ld_x32(tO + ch * 32, orr);
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
+            if (in_range) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        }
+        if (in_range) {
+          if (p.acc_o != nullptr)
+            p.acc_lse[row_idx] = lse_out;
+          else
+            p.lse[row_idx] = lse_out;
+        }
+      }
+
     }
   }
 

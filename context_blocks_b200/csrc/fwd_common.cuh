@@ -29,6 +29,8 @@ constexpr int kAccFinal = 2;   // write the bf16 output instead of the fp32 stat
 struct FwdParams {
   __nv_bfloat16* o;     // [B*H, Nq, D]
   float* lse;           // [B*H, Nq]
+  int items;            // work items: B*H * blocks_per_bh
+  int blocks_per_bh;    // query blocks of kQTiles * kBM rows per (b, h)
   int Nq;
   int Nk;               // keys in all chunks of the launch
   int n_kv_tiles;       // key tiles in all chunks of the launch

@@ -236,7 +236,13 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   prm.acc_o = acc.acc_o;
   prm.acc_lse = acc.acc_lse;
   prm.acc_flags = acc.flags;
-  dim3 grid((Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM), BH);
+  // Persistent grid: one CTA per SM (shared memory and tensor memory allow
+  // no more), each walking the (b*h, 256-row block) items.
+  prm.blocks_per_bh = (Nq + pa::kQTiles * pa::kBM - 1) / (pa::kQTiles * pa::kBM);
+  const long long items = static_cast<long long>(prm.blocks_per_bh) * BH;
+  if (items > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many query blocks");
+  prm.items = static_cast<int>(items);
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(items, st->sm_count));
   kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, kv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
