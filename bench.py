@@ -49,13 +49,21 @@ UNIT = "TFLOPS"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic of one attn_fwd launch on the default workload, from an ncu
-# capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
-# kernel source whose digest is recorded with it.  See profiles/.
+# DRAM traffic of one attn_fwd launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) from ncu captures, valid only for the kernel source
+# whose digest is recorded with them.  The HunyuanVideo figure is a 4-head
+# capture of the same sequence shape scaled to 24 heads (every head's items
+# are alike, so traffic grows in proportion to heads).  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "c04f091c8d0496fe9c6bf43b9be3785dd74a359bc103c5c2b6d94497361b1e65",
-    "bytes_per_launch": 84987392 + 5752576,   # dram__bytes_read.sum + dram__bytes_write.sum
-    "capture": "ncu --set full, FLUX shape, bench.py --steps 20 --warmup 5 --no-extra --no-cpu-baseline",
+    "source_sha256": "30c27aa91acc67998a5ca7492ba9e4faa927ee5730e92690d35d50b8c1cc0754",
+    "bytes_per_launch": {
+        "hunyuan": (984587776 + 124680192) * 24 // 4,
+        "flux": 85081856 + 4751872,
+    },
+    "capture": {
+        "hunyuan": "ncu --set full, bench.py --heads 4 --steps 3 --warmup 3 --no-extra --no-cpu-baseline, x 24/4",
+        "flux": "ncu --set full, bench.py --workload flux --steps 20 --warmup 5 --no-extra --no-cpu-baseline",
+    },
 }
 
 
@@ -544,9 +552,9 @@ def run_ours(args):
     fl_launch = fl / len(w.chunks)
     achieved = fl_launch / (fwd_mean_ms * 1e-3) / 1e12
     traffic = None
-    if (not fp8 and w.name == "flux" and w.H == workloads.get("flux").H
-            and NCU_TRAFFIC["source_sha256"] == _kernel_digest()):
-        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    if (not fp8 and len(w.chunks) == 1 and w.name in NCU_TRAFFIC["bytes_per_launch"]
+            and w.H == workloads.get(w.name).H and NCU_TRAFFIC["source_sha256"] == _kernel_digest()):
+        traffic = NCU_TRAFFIC["bytes_per_launch"][w.name]
     # e4m3 contractions: the measured bf16 peak times the nominal e4m3/bf16 ratio of 2
     peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
     alg_bytes = workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk // len(w.chunks), w.d)

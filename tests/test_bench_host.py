@@ -143,3 +143,11 @@ def test_heads_override_keeps_the_sequence_shape():
     h = workloads.get("hunyuan")
     assert (w.H, w.Nq, w.Nk, w.d, w.chunks) == (4, h.Nq, h.Nk, h.d, h.chunks)
     assert bench._workload(argparse.Namespace(workload="flux", heads=None)) == workloads.get("flux")
+
+
+def test_ring_shard_sizes_cover_the_sequence():
+    for n, world in ((119056, 8), (4608, 3), (4481, 4), (5, 8), (7, 1)):
+        sizes = bench.shard_sizes(n, world)
+        assert len(sizes) == world and sum(sizes) == n
+        assert max(sizes) - min(sizes) <= 1
+        assert sizes == sorted(sizes, reverse=True)
