@@ -122,10 +122,13 @@ def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
         if s < world - 1:
             nb = kv_lens[ent["recv_block"]]
             nxt = (view(bufs[ent["recv_buffer"]][0], nb), view(bufs[ent["recv_buffer"]][1], nb))
-            ops = [dist.P2POp(dist.isend, cur_k, ent["send_to"], group),
-                   dist.P2POp(dist.isend, cur_v, ent["send_to"], group),
-                   dist.P2POp(dist.irecv, nxt[0], ent["recv_from"], group),
-                   dist.P2POp(dist.irecv, nxt[1], ent["recv_from"], group)]
+            # P2POp takes global ranks; the schedule is in ranks of the group.
+            to_rank = ent["send_to"] if group is None else dist.get_global_rank(group, ent["send_to"])
+            from_rank = ent["recv_from"] if group is None else dist.get_global_rank(group, ent["recv_from"])
+            ops = [dist.P2POp(dist.isend, cur_k, to_rank, group),
+                   dist.P2POp(dist.isend, cur_v, to_rank, group),
+                   dist.P2POp(dist.irecv, nxt[0], from_rank, group),
+                   dist.P2POp(dist.irecv, nxt[1], from_rank, group)]
             if cuda:
                 with torch.cuda.stream(comm):
                     # The buffer being received into held the block of step

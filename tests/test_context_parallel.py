@@ -76,6 +76,46 @@ def _ring_rank(rank, world, port, q_lens, kv_lens, gather, out_q):
         dist.destroy_process_group()
 
 
+def _subgroup_rank(rank, world, port, out_q):
+    """Ranks 0 and 2 of a 3-rank world run the ring in a subgroup; rank 1 only
+    joins the group creation (a collective over the world)."""
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import ring_attention
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        sub = dist.new_group([0, 2])
+        if rank == 1:
+            out_q.put((rank, 0.0, 0.0, []))
+            return
+        me = 0 if rank == 0 else 1
+        q, k, v = _global_case(7, 1, 2, 10, 8)
+        lens = (4, 6)
+        s0 = 0 if me == 0 else 4
+        sl = slice(s0, s0 + lens[me])
+        o = torch.empty((1, 2, lens[me], 8), dtype=torch.float64)
+        lse = torch.empty((1, 2, lens[me]), dtype=torch.float64)
+
+        def attend(qq, kk, vv, o_acc, lse_acc, first, final, out, scale):
+            _oracle_fold(qq, kk, vv, o, lse, first, final, out, scale)
+
+        trace = []
+        out, _ = ring_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(), group=sub,
+                                scale=SCALE, out=torch.empty_like(o), attend=attend, trace=trace)
+        o_ref, l_ref = oracle.attention(q[:, :, sl], k, v, SCALE)
+        out_q.put((rank, float(np.abs(out.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()), trace))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_ring_attention_in_a_subgroup():
+    got = _run(_subgroup_rank, 3)
+    for rank in (0, 2):
+        err_o, err_l, trace = got[rank]
+        assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
+        assert len(trace) == 2
+
+
 def _run(target, world, *args):
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
