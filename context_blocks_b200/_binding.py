@@ -108,8 +108,13 @@ def _check(rc: int, where: str, check: bool = False) -> None:
 
 
 def _stream_handle(stream, device) -> int:
+    """cudaStream_t of `stream`, or of torch's current stream on `device`."""
     import torch
     if stream is None:
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:  # the handle alone, without building a Stream object
+            index = device.index if isinstance(device, torch.device) else device
+            return int(raw(torch.cuda.current_device() if index is None else int(index)))
         stream = torch.cuda.current_stream(device)
     if isinstance(stream, int):
         return stream
