@@ -537,8 +537,8 @@ def run_ours(args):
     peaks = _peaks()
     sampler = ClockSampler(local)
     fp8 = bool(getattr(args, "fp8", False))
-    if ws > 1 and args.parallel == "ring":
-        return run_ring(args, pa, w, peaks, sampler, device, barrier)
+    if ws > 1 and args.parallel in ("ring", "ulysses"):
+        return run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=(args.parallel == "ulysses"))
     res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier, fp8=fp8)
     if res["status"] != 0:
         raise SystemExit(f"device status {res['status']} after the timed region")
@@ -608,11 +608,13 @@ def shard_sizes(n: int, world: int):
     return [n // world + (1 if r < n % world else 0) for r in range(world)]
 
 
-def run_ring(args, pa, w, peaks, sampler, device, barrier):
-    """Ring Attention over the process group: rank r holds shard r of the
-    query rows and of the K/V rows of workload `w` and runs
-    context_parallel.ring_attention.  Value = the whole problem's FLOPs per
-    step over the slowest rank's time (strong scaling)."""
+def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False):
+    """Context parallelism over the process group: rank r holds shard r of
+    the query rows and of the K/V rows of workload `w` and runs
+    context_parallel.ring_attention (or, with ``ulysses``, the all-to-all
+    form, which needs equal shards and heads divisible by the rank count).
+    Value = the whole problem's FLOPs per step over the slowest rank's time
+    (strong scaling)."""
     import dataclasses
 
     import torch
@@ -621,6 +623,8 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier):
 
     ws, rank = dist.get_world_size(), dist.get_rank()
     nq_all, nk_all = shard_sizes(w.Nq, ws), shard_sizes(w.Nk, ws)
+    if ulysses and (len(set(nq_all)) > 1 or nq_all != nk_all or w.H % ws):
+        raise SystemExit(f"--parallel ulysses needs Nq = Nk divisible by {ws} and heads divisible by {ws}")
     wr = dataclasses.replace(w, Nq=nq_all[rank], Nk=nk_all[rank], chunks=(nk_all[rank],), seed=w.seed + 100 * rank)
     q, k, v = workloads.make_case(wr, device=device)
     out = torch.empty_like(q)
@@ -632,7 +636,15 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier):
         pa.attn_fwd_accum(qq, kk, vv, o_acc, lse_acc, first=first, final=final, out=o, scale=scale)
         fwd_ev[1].append(_record())
 
+    def attend_full_timed(qq, kk, vv, scale):
+        fwd_ev[0].append(_record())
+        res = pa.attn_fwd(qq, kk, vv, scale=scale)
+        fwd_ev[1].append(_record())
+        return res
+
     def step(timed=False):
+        if ulysses:
+            return cp.ulysses_attention(q, k, v, scale=w.scale, attend_full=attend_full_timed if timed else None)
         return cp.ring_attention(q, k, v, kv_lens=nk_all, scale=w.scale, out=out, comm_stream=comm,
                                  attend=attend_timed if timed else None)
 
@@ -659,10 +671,14 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier):
     # the fold kernel: this rank's FLOPs per ring pass over its launches
     fl_rank = workloads.flops(w.B, w.H, nq_all[rank], w.Nk, w.d)
     launch_ms = statistics.fmean(fwd_ms)
-    achieved = fl_rank / ws / (launch_ms * 1e-3) / 1e12
+    # ring: one fold launch per block, 1/ws of the rank's FLOPs each; Ulysses:
+    # one launch over the rank's heads and the whole sequence
+    achieved = (fl_rank / ws if not ulysses else fl_rank) / (launch_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": None, "kernel": f"attn_fwd_kernel<{w.d}, false> (accumulate mode)", "launch_ms": launch_ms,
+            "traffic": None,
+            "kernel": f"attn_fwd_kernel<{w.d}, false>" + ("" if ulysses else " (accumulate mode)"),
+            "launch_ms": launch_ms,
             "peak_basis": f"{peaks['source']} burst bf16 (MEASURED_PEAKS.json bf16_tflops), rank {rank}"}
     # End to end: each step uploads this rank's shards from pinned host
     # memory, runs the ring, downloads this rank's output and LSE.
@@ -692,11 +708,12 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(_config(w, parallelism=f"ring attention over {ws} ranks (NCCL P2P on a second stream)"),
+            "config": dict(_config(w, parallelism=(f"Ulysses attention over {ws} ranks (two NCCL all-to-alls)" if ulysses
+                                                   else f"ring attention over {ws} ranks (NCCL P2P on a second stream)")),
                            q_shards=nq_all, kv_shards=nk_all,
                            l2="each rank's K/V blocks rotate through the ring; inputs far larger than L2"),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak, "roofline": roof, "clocks": sampler.summary(),
-            "gpu_launches": args.steps * ws,
+            "gpu_launches": args.steps * (1 if ulysses else ws),
             "e2e": {"value": fl * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
                     "d2h_bytes_per_step": int(out.numel() * 2 + out.numel() // w.d * 4), "steps": e_steps,
@@ -726,19 +743,23 @@ class ModeSets:
             del k, v
             st = {"q": q, "k": [a for a, _ in pairs], "v": [b for _, b in pairs], "o": torch.empty_like(q),
                   "lse": torch.empty(q.shape[:3], dtype=torch.float32, device=device)}
-            if mode == "chunks" and n > 1:
+            if mode in ("chunks", "fwds") and n > 1:
                 st["o_parts"] = torch.empty((n,) + tuple(q.shape), dtype=torch.bfloat16, device=device)
                 st["lse_parts"] = torch.empty((n,) + tuple(q.shape[:3]), dtype=torch.float32, device=device)
             if mode == "fold":
                 st["o_acc"] = torch.empty(q.shape, dtype=torch.float32, device=device)
             self.sets.append(st)
-        self.launches = {"chunks": n + (1 if n > 1 else 0), "fused": 1, "fold": n}[mode]
+        self.launches = {"chunks": n + (1 if n > 1 else 0), "fwds": n, "fused": 1, "fold": n}[mode]
 
     def run(self, i):
         pa, w, st = self.pa, self.w, self.sets[i % len(self.sets)]
         if self.mode == "chunks":
             pa.blockwise_attention(st["q"], st["k"], st["v"], scale=w.scale, o_parts=st.get("o_parts"),
                                    lse_parts=st.get("lse_parts"), out=st["o"], lse=st["lse"])
+        elif self.mode == "fwds":  # the per-chunk forwards alone, into the partial buffers
+            for c in range(len(st["k"])):
+                pa.attn_fwd(st["q"], st["k"][c], st["v"][c], scale=w.scale, out=st["o_parts"][c],
+                            lse=st["lse_parts"][c])
         elif self.mode == "fused":
             pa.attn_fwd_chunks(st["q"], st["k"], st["v"], scale=w.scale, out=st["o"], lse=st["lse"])
         else:
@@ -795,7 +816,8 @@ def mode_timing(pa, w, mode, steps, warmup, device, graph=False):
     torch.cuda.empty_cache()
     fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
     return {"step_ms": ms, "tflops_step": fl / (ms * 1e-3) / 1e12, "launches_per_step":
-            {"chunks": len(w.chunks) + (1 if len(w.chunks) > 1 else 0), "fused": 1, "fold": len(w.chunks)}[mode],
+            {"chunks": len(w.chunks) + (1 if len(w.chunks) > 1 else 0), "fwds": len(w.chunks), "fused": 1,
+             "fold": len(w.chunks)}[mode],
             "timing": "CUDA graph replay" if graph else "eager launches"}
 
 
@@ -852,7 +874,7 @@ def extra_measurements(pa, device, peaks):
             ent["merge_gbs"] = mb / (ent["merge_ms"] * 1e-3) / 1e9
         ent["pct_of_bf16_peak"] = 100.0 * ent["fwd_tflops"] / peaks["bf16_tflops"]
         out[name] = ent
-        for mode in ("chunks", "fused", "fold"):
+        for mode in ("fwds", "chunks", "fused", "fold"):
             g = mode_timing(pa, w, mode, 200, 3, device, graph=True)
             g["frac_of_bf16_peak"] = g["tflops_step"] / peaks["bf16_tflops"]
             out[f"{name}_{mode}_graph"] = g
@@ -908,8 +930,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="hunyuan", choices=sorted(workloads.WORKLOADS))
-    ap.add_argument("--parallel", choices=["ring", "replicas"], default="ring",
-                    help="with more than one GPU: ring attention over the ranks, or independent replicas")
+    ap.add_argument("--parallel", choices=["ring", "ulysses", "replicas"], default="ring",
+                    help="with more than one GPU: ring or Ulysses attention over the ranks, or independent replicas")
     ap.add_argument("--fp8", action="store_true",
                     help="time the e4m3 forward (pa_attn_fwd_fp8) instead of bf16; one-chunk workloads")
     ap.add_argument("--heads", type=int, default=None,
