@@ -30,7 +30,7 @@
 // warpgroup hands P to the MMA warp in two halves, so P.V on the first 64
 // keys starts while the second half is still being computed.
 //
-// Accumulate mode (FwdParams::acc_o set): the launch folds its chunk into a
+// Accumulate mode (kAcc; FwdParams::acc_o and acc_lse set): the launch folds its chunk into a
 // caller-owned running state, a normalised fp32 O and its LSE.  That state is
 // exactly (O_unnormalised = O, l = 1, m = LSE * log2(e)) in the online softmax
 // below, so the softmax threads load it into the O accumulator before the
@@ -94,7 +94,11 @@ struct FwdLayout {
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // one 128-row tile of Q, K or V
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kQTiles * kTileBytes;
-  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  // One 4 KB staging area per softmax warp: 32 rows x 128 bytes of O (or of
+  // the fp32 running state) on their way between TMEM and global memory.
+  static constexpr int kStageOff = kRingOff + kStages * kTileBytes;
+  static constexpr int kStageWarpBytes = 32 * 128;
+  static constexpr int kBarOff = kStageOff + 8 * kStageWarpBytes;
   // q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain,
   // p_part[2][3] (parts of P before the last, which arrives on p_full), q_empty
   static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 6 + 1;
@@ -109,7 +113,111 @@ struct FwdLayout {
       (kBytes + 1024 > kMinOneCtaPerSm) ? (kBytes + 1024) : kMinOneCtaPerSm;
 };
 
-template <int D, bool kFp8 = false>
+// O rows move between TMEM and global memory through a 4 KB staging area per
+// warp, 128 bytes of each of the warp's 32 rows at a time.  A thread holds one
+// row (its TMEM lane); it writes or reads its row's piece in the staging area
+// with 16-byte chunk c of row r at chunk position c ^ (r % 8), so that 8
+// consecutive rows fall in distinct banks, while global memory sees 4 rows x
+// 128 contiguous bytes per warp instruction instead of 32 separate rows.
+// Both helpers stay out of line: they run once per work item, and inlined
+// into the kernel they cost the key loop registers.
+//
+// Global rows: row r of the warp is at dst0 + r * D elements; rows
+// r >= rows_left are neither read nor written.
+
+// Scale this thread's O row (TMEM columns [tO, tO + D)) by inv_l and store it:
+// bf16 to `o_bf16`, or, when o_bf16 is null, fp32 to `o_f32`.
+template <int D>
+__device__ __noinline__ void store_o_rows(uint32_t tO, uint32_t stg, __nv_bfloat16* o_bf16, float* o_f32,
+                                          int rows_left, float inv_l) {
+  const int lane = threadIdx.x % 32;
+  const int r0 = lane >> 3, c = lane & 7;
+  auto stage4 = [&](int c0, const uint32_t (&w)[16]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      st_shared_v4(stg + lane * 128 + (((c0 + u) ^ (lane & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2],
+                   w[4 * u + 3]);
+  };
+  auto drain = [&](uint8_t* dst, int row_bytes) {
+    dst += r0 * row_bytes + c * 16;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int r = 4 * k + r0;
+      const uint4 x = ld_shared_v4(stg + r * 128 + ((c ^ (r & 7)) << 4));
+      if (r < rows_left) *reinterpret_cast<uint4*>(dst + k * 4 * row_bytes) = x;
+    }
+  };
+  if (o_bf16 != nullptr) {
+#pragma unroll 1
+    for (int h = 0; h < D / 64; ++h) {  // 64 bf16 columns = 128 bytes a piece
+      __syncwarp();                      // the previous piece has left the staging area
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t orr[32], pk[16];
+        tmem_ld_x32(tO + h * 64 + hh * 32, orr);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
+        stage4(4 * hh, pk);
+      }
+      __syncwarp();
+      drain(reinterpret_cast<uint8_t*>(o_bf16 + h * 64), D * 2);
+    }
+  } else {
+#pragma unroll 1
+    for (int ch = 0; ch < D / 32; ++ch) {  // 32 fp32 columns = 128 bytes a piece
+      uint32_t orr[32];
+      tmem_ld_x32(tO + ch * 32, orr);
+      __syncwarp();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(orr[16 * hh + e]) * inv_l);
+        stage4(4 * hh, w);
+      }
+      __syncwarp();
+      drain(reinterpret_cast<uint8_t*>(o_f32 + ch * 32), D * 4);
+    }
+  }
+}
+
+// Load this thread's fp32 row of a running state into TMEM columns
+// [tO, tO + D) (zeros where `have` is false); waits for the TMEM stores.
+template <int D>
+__device__ __noinline__ void load_state_rows(uint32_t tO, uint32_t stg, const float* src0, int rows_left, bool have) {
+  const int lane = threadIdx.x % 32;
+  const int r0 = lane >> 3, c = lane & 7;
+#pragma unroll 1
+  for (int ch = 0; ch < D / 32; ++ch) {
+    __syncwarp();  // the previous piece has left the staging area
+    const uint4* src = reinterpret_cast<const uint4*>(src0 + r0 * D + ch * 32) + c;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int r = 4 * k + r0;
+      uint4 x = make_uint4(0u, 0u, 0u, 0u);
+      if (r < rows_left) x = __ldg(src + k * 4 * (D / 4));
+      st_shared_v4(stg + r * 128 + ((c ^ (r & 7)) << 4), x.x, x.y, x.z, x.w);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t w[16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint4 x = ld_shared_v4(stg + lane * 128 + (((4 * hh + u) ^ (lane & 7)) << 4));
+        w[4 * u] = have ? x.x : 0u;
+        w[4 * u + 1] = have ? x.y : 0u;
+        w[4 * u + 2] = have ? x.z : 0u;
+        w[4 * u + 3] = have ? x.w : 0u;
+      }
+      tmem_st_x16(tO + ch * 32 + hh * 16, w);
+    }
+  }
+  tmem_st_wait();
+}
+
+template <int D, bool kFp8 = false, bool kAcc = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ KvChunks kv,
                     const FwdParams p) {
@@ -290,7 +398,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     };
     // With a running state loaded into O (accumulate mode) even the first
     // P.V accumulates.
-    const bool o_loaded = (p.acc_o != nullptr) && !(p.acc_flags & kAccFirst);
+    const bool o_loaded = kAcc && !(p.acc_flags & kAccFirst);
 
     bool ok = true;
     int idx = 0;  // ring position (over all items)
@@ -402,7 +510,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         o_mul = p.o_scale;
       }
     }
-    const bool o_loaded = (p.acc_o != nullptr) && !(p.acc_flags & kAccFirst);
+    const bool o_loaded = kAcc && !(p.acc_flags & kAccFirst);
     bool ok = true;
     int g = 0;   // key tiles over all items: phases of the S barrier
     int it = 0;  // items of this CTA: phase of the O barrier
@@ -420,29 +528,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // key seen yet) start empty, with O = 0.  (This warpgroup's epilogue of
       // the previous item has read O out; its P V are complete.)
       if (o_loaded) {
-        const bool in_range = row_of(item) < p.Nq;
-        const size_t row_idx = index_of(item);
-        const float lse0 = in_range ? p.acc_lse[row_idx] : -INFINITY;
+        const int row0 = row_of(item) - lane;  // first row of this warp's 32
+        const size_t idx0 = index_of(item) - lane;
+        const float lse0 = (row0 + lane < p.Nq) ? p.acc_lse[idx0 + lane] : -INFINITY;
         const bool have = lse0 > -INFINITY;
         if (have) {
           m_ref = lse0 * 1.4426950408889634f;
           l = 1.f;
         }
-        const float4* src = reinterpret_cast<const float4*>(p.acc_o + row_idx * D);
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t orr[32];
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float4 x = have ? __ldg(src + ch * 8 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-            orr[4 * v] = __float_as_uint(x.x);
-            orr[4 * v + 1] = __float_as_uint(x.y);
-            orr[4 * v + 2] = __float_as_uint(x.z);
-            orr[4 * v + 3] = __float_as_uint(x.w);
-          }
-          tmem_st_x32(tO + ch * 32, orr);
-        }
-        tmem_st_wait();
+        load_state_rows<D>(tO, base + L::kStageOff + warp * L::kStageWarpBytes, p.acc_o + idx0 * D, p.Nq - row0, have);
       }
 
       for (int j = 0; j < n; ++j, ++g) {
@@ -559,52 +653,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (ok) {
         tc_fence_after();
-        const bool in_range = row_of(item) < p.Nq;
-        const size_t row_idx = index_of(item);
-        const float inv_l = o_mul / l;
+        const int row0 = row_of(item) - lane;  // first row of this warp's 32
+        const size_t idx0 = index_of(item) - lane;
         const float lse_out = (m_ref + lg2_approx(l)) * 0.69314718055994531f;
-        const bool state_out = (p.acc_o != nullptr) && !(p.acc_flags & kAccFinal);
-        if (state_out) {
-          // Running state: normalised fp32 O and its LSE.
-          float4* dst = reinterpret_cast<float4*>(p.acc_o + row_idx * D);
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t orr[32];
-            tmem_ld_x32(tO + ch * 32, orr);
-            if (in_range) {
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[ch * 8 + v] = make_float4(__uint_as_float(orr[4 * v]) * inv_l, __uint_as_float(orr[4 * v + 1]) * inv_l,
-                                              __uint_as_float(orr[4 * v + 2]) * inv_l,
-                                              __uint_as_float(orr[4 * v + 3]) * inv_l);
-            }
-          }
-        } else {
-          __nv_bfloat16* orow = p.o + row_idx * D;
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t orr[32];
-            tmem_ld_x32(tO + ch * 32, orr);
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
-            if (in_range) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-            }
-          }
-        }
-        if (in_range) {
-          if (p.acc_o != nullptr)
-            p.acc_lse[row_idx] = lse_out;
-          else
-            p.lse[row_idx] = lse_out;
-        }
+        // bf16 output, or (accumulate mode, before the final fold) the
+        // running state: normalised fp32 O.
+        const bool state_out = kAcc && !(p.acc_flags & kAccFinal);
+        store_o_rows<D>(tO, base + L::kStageOff + warp * L::kStageWarpBytes, state_out ? nullptr : p.o + idx0 * D,
+                        kAcc ? p.acc_o + idx0 * D : nullptr, p.Nq - row0, o_mul / l);
+        if (row0 + lane < p.Nq) (kAcc ? p.acc_lse : p.lse)[idx0 + lane] = lse_out;
       }
-
     }
   }
 

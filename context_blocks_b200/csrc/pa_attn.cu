@@ -73,7 +73,7 @@ struct DeviceState {
   int sm_count = 0;
   int* status = nullptr;  // device address of pa::g_status
   unsigned char* noalloc_scratch = nullptr;  // device address of pa::g_noalloc_scratch
-  bool fwd_attr[3] = {false, false, false};  // d = 64, d = 128, e4m3 d = 128
+  bool fwd_attr[5] = {};  // d = 64, d = 128, e4m3 d = 128, accumulate d = 64, accumulate d = 128
 };
 
 
@@ -209,8 +209,14 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   }
   kv.n_chunks = n_chunks;
   if (nk_total > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "more than 2^31 keys in one call");
-  auto kern = pa::single::attn_fwd_kernel<D, kFp8>;
-  const int slot = kFp8 ? 2 : (D == 64) ? 0 : 1;
+  // Accumulate mode is its own instantiation (bf16 only), so that the plain
+  // forward carries none of its code.
+  const bool accum = acc.acc_o != nullptr;
+  if (kFp8 && accum) return fail(PA_ERR_UNSUPPORTED, "accumulate mode takes bf16 inputs");
+  auto kern = pa::single::attn_fwd_kernel<D, kFp8, false>;
+  if constexpr (!kFp8)
+    if (accum) kern = pa::single::attn_fwd_kernel<D, false, true>;
+  const int slot = kFp8 ? 2 : (D == 64 ? 0 : 1) + (accum ? 3 : 0);
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!st->fwd_attr[slot]) {

@@ -258,6 +258,16 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// 16-byte shared-memory store and load (addresses 16-byte aligned).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
 // Two floats to two e4m3 bytes, round to nearest even, saturating at +-448:
 // `hi` goes to the upper byte.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
