@@ -63,6 +63,11 @@ constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms; the wait itself stays bou
 constexpr int kPParts = 2;         // P is handed to the MMA warp in this many parts
 constexpr int kStages = 4;         // K/V ring slots (each holds one K or one V tile)
 constexpr int kMaxChunks = 8;      // K/V chunks one launch can consume
+// With e4m3 inputs the tensor pipe needs half the time of the exponentials,
+// so pairs e of each 32-key chunk whose bit is set here (3 in 8) take 2^x on
+// the FMA pipe (exp2_poly2_x2) instead of MUFU.  Measured: 1/4 and 1/2 are
+// slower than 3/8; in the bf16 path any share is slower.
+constexpr uint32_t kPolyPairsFp8 = 0xA4A4u;
 
 // The K/V chunks of one launch: keys are the concatenation of the chunks, in
 // order; each chunk has its own tensor maps and its own (possibly ragged)
@@ -593,8 +598,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_st_x32(tO + ch * 32, orr);
           }
         }
-        // x = s * c - m_ref on packed pairs, P = 2^x on MUFU, the row sum in
-        // four packed partial sums.
+        // x = s * c - m_ref on packed pairs, P = 2^x on MUFU (with e4m3
+        // inputs 3 pairs in 8 on the FMA pipe instead), the row sum in four
+        // packed partial sums.
         const float neg_m = -m_ref;
         const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
         uint64_t l4[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
@@ -603,10 +609,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float x0, x1;
-            f2_split(f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2), x0, x1);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
+            const uint64_t x2 = f2_fma(f2(s[ch * 32 + 2 * e], s[ch * 32 + 2 * e + 1]), c2, nm2);
+            float p0, p1;
+            if (kFp8 && ((kPolyPairsFp8 >> e) & 1)) {
+              f2_split(exp2_poly2_x2(x2), p0, p1);
+            } else {
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             l4[e & 3] = f2_add(l4[e & 3], f2(p0, p1));
             if constexpr (kFp8) {
               // four e4m3 keys per 32-bit column, lowest key in the low byte

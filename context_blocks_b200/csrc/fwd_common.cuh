@@ -94,4 +94,35 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
+
+// 2^x on the FMA pipe for both halves of a pair, to take load off the MUFU
+// unit in the e4m3 path (whose P is rounded to e4m3 right after).  Cody-Waite
+// range reduction x = n + f, n = round-to-nearest(x) by adding and subtracting
+// 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by a degree-2 polynomial minimax in
+// relative error (1.73e-3; coefficients from gen_exp2_poly.py); 2^n by adding
+// n to the exponent field.  x is clamped to >= -126 so that the exponent add
+// cannot reach the sign bit (masked keys, x = -inf, give ~2^-126, which
+// rounds to 0 in e4m3).
+constexpr float kExp2P2C0 = 1.000443101e+00f;
+constexpr float kExp2P2C1 = 7.034479976e-01f;
+constexpr float kExp2P2C2 = 2.384289354e-01f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t exp2_poly2_x2(uint64_t x) {
+  float a, b;
+  f2_split(x, a, b);
+  const uint64_t xc = f2(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const uint64_t t = f2_add(xc, f2(kRoundMagic, kRoundMagic));   // magic + n
+  const uint64_t n = f2_add(t, f2(-kRoundMagic, -kRoundMagic));  // n (exact)
+  const uint64_t fr = f2_fma(n, f2(-1.f, -1.f), xc);             // f = x - n (exact)
+  uint64_t p = f2_fma(f2(kExp2P2C2, kExp2P2C2), fr, f2(kExp2P2C1, kExp2P2C1));
+  p = f2_fma(p, fr, f2(kExp2P2C0, kExp2P2C0));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  // the low bits of t hold n; shifted by 23 they land in the exponent field
+  return f2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+            __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
 }  // namespace pa
