@@ -55,10 +55,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of the same sequence shape scaled to 24 heads (every head's items
 # are alike, so traffic grows in proportion to heads).  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "30c27aa91acc67998a5ca7492ba9e4faa927ee5730e92690d35d50b8c1cc0754",
+    "source_sha256": "27869241fc8cb349bf30173a3896eeb6bae6e7fa39a278c5d26f738e22be35e3",
     "bytes_per_launch": {
-        "hunyuan": (984587776 + 124680192) * 24 // 4,
-        "flux": 85081856 + 4751872,
+        "hunyuan": (1007819520 + 124523264) * 24 // 4,
+        "flux": 85010432 + 5947648,
     },
     "capture": {
         "hunyuan": "ncu --set full, bench.py --heads 4 --steps 3 --warmup 3 --no-extra --no-cpu-baseline, x 24/4",
