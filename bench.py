@@ -271,11 +271,22 @@ class Step:
                 merge_events[1].append(_record())
 
 
+_EVENT_POOL = []
+
+
 def _record():
+    """Record a timing event on the current stream.  Events come from a pool
+    made before the timed region (_event_pool), so that creating them does
+    not add host time between the launches being timed."""
     import torch
-    e = torch.cuda.Event(enable_timing=True)
+    e = _EVENT_POOL.pop() if _EVENT_POOL else torch.cuda.Event(enable_timing=True)
     e.record()
     return e
+
+
+def _event_pool(n: int) -> None:
+    import torch
+    _EVENT_POOL[:] = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
 
 
 def _sets_for(w: workloads.Workload, fp8: bool = False) -> int:
@@ -295,6 +306,7 @@ def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, fp8=
     torch.cuda.synchronize()
     fwd_ev = ([], [])
     mrg_ev = ([], [])
+    _event_pool(2 * steps * st.launches_per_step)
     if barrier:
         barrier()
     torch.cuda.synchronize()

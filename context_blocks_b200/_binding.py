@@ -64,6 +64,8 @@ _lock = threading.Lock()
 def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     """Load (once) and return the library; raises if it is not built."""
     global _lib
+    if path is None and _lib is not None:  # the common case, without the lock
+        return _lib
     with _lock:
         if _lib is not None and path is None:
             return _lib
@@ -107,14 +109,19 @@ def _check(rc: int, where: str, check: bool = False) -> None:
             raise PaError(code, where, "reported by the device after the call")
 
 
+_raw_stream = None  # torch's current-stream handle getter, looked up once
+
+
 def _stream_handle(stream, device) -> int:
     """cudaStream_t of `stream`, or of torch's current stream on `device`."""
+    global _raw_stream
     import torch
     if stream is None:
-        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
-        if raw is not None:  # the handle alone, without building a Stream object
+        if _raw_stream is None:
+            _raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", False)
+        if _raw_stream:  # the handle alone, without building a Stream object
             index = device.index if isinstance(device, torch.device) else device
-            return int(raw(torch.cuda.current_device() if index is None else int(index)))
+            return int(_raw_stream(torch.cuda.current_device() if index is None else int(index)))
         stream = torch.cuda.current_stream(device)
     if isinstance(stream, int):
         return stream
@@ -127,7 +134,7 @@ def _check_bf16(name, t, ndim):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != torch.bfloat16:
         raise TypeError(f"{name} must be bfloat16 (got {t.dtype})")
-    if t.device.type != "cuda":
+    if not t.is_cuda:
         raise ValueError(f"{name} must live on a CUDA device")
     if t.dim() != ndim or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
@@ -144,9 +151,9 @@ def attn_fwd(q, k, v, scale: Optional[float] = None, out=None, lse=None, stream=
     _check_bf16("k", k, 4)
     _check_bf16("v", v, 4)
     B, H, Nq, d = q.shape
-    if k.shape[:2] != (B, H) or k.shape[3] != d or v.shape != k.shape:
+    kB, kH, Nk, kd = k.shape
+    if kB != B or kH != H or kd != d or v.shape != k.shape:
         raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
-    Nk = k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out, lse = _outputs(q, out, lse)
