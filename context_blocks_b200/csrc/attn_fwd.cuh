@@ -30,15 +30,20 @@
 // warpgroup hands P to the MMA warp in two halves, so P.V on the first 64
 // keys starts while the second half is still being computed.
 //
-// Accumulate mode (kAcc; FwdParams::acc_o and acc_lse set): the launch folds its chunk into a
-// caller-owned running state, a normalised fp32 O and its LSE.  That state is
+// Accumulate mode (kAcc; FwdParams::acc_o and acc_lse set): the launch folds
+// its chunk into a caller-owned running state, a normalised fp32 O and its
+// LSE.  That state is
 // exactly (O_unnormalised = O, l = 1, m = LSE * log2(e)) in the online softmax
 // below, so the softmax threads load it into the O accumulator before the
 // first tile and carry on; the epilogue writes the updated state back (or,
 // on the final fold, the bf16 output).
 //
 // With kFp8 the same kernel takes e4m3 Q, K, V (per-tensor scales folded into
-// the logit scale and the epilogue) and issues kind::f8f6f4 MMAs.
+// the logit scale and the epilogue) and issues kind::f8f6f4 MMAs; 3 in 8 of
+// its exponentials are computed on the FMA pipe (exp2_poly2_x2).
+//
+// Shared memory: Q (two tiles), a 4-slot K/V ring, a 4 KB output staging area
+// per softmax warp, then the barriers (230.6 KB with bf16 d = 128).
 //
 // Online softmax in base 2: x = s * scale * log2(e).  m_ref is the reference
 // maximum the exponentials of this row use; it moves only when a new tile's
