@@ -92,6 +92,13 @@ def _workload(args):
     return w
 
 
+def _basis(peaks) -> str:
+    """Where the peak figures came from, for the JSON line."""
+    if peaks["source"] == "measured":
+        return "measured burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
+    return "fallback burst bf16 of the profiling recipe (MEASURED_PEAKS.json absent on this machine)"
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -574,8 +581,8 @@ def run_ours(args):
         alg_bytes -= (w.Nq + 2 * (w.Nk // len(w.chunks))) * w.d * w.B * w.H
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic,
-            "kernel": f"attn_fwd_kernel<{w.d}, {'true' if fp8 else 'false'}>", "launch_ms": fwd_mean_ms,
-            "peak_basis": (f"{peaks['source']} burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
+            "kernel": f"attn_fwd_kernel<{w.d}, {'true' if fp8 else 'false'}, false>", "launch_ms": fwd_mean_ms,
+            "peak_basis": (_basis(peaks)
                            + (" x 2, the nominal e4m3/bf16 ratio" if fp8 else "")
                            + f"; frac of sustained {achieved / (peak * peaks['bf16_tflops_sustained'] / peaks['bf16_tflops']):.3f}"),
             "algorithmic_bytes_per_launch": alg_bytes}
@@ -689,9 +696,9 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False):
     peak = peaks["bf16_tflops"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": None,
-            "kernel": f"attn_fwd_kernel<{w.d}, false>" + ("" if ulysses else " (accumulate mode)"),
+            "kernel": f"attn_fwd_kernel<{w.d}, false, {'false' if ulysses else 'true'}>",
             "launch_ms": launch_ms,
-            "peak_basis": f"{peaks['source']} burst bf16 (MEASURED_PEAKS.json bf16_tflops), rank {rank}"}
+            "peak_basis": f"{_basis(peaks)}, rank {rank}"}
     # End to end: each step uploads this rank's shards from pinned host
     # memory, runs the ring, downloads this rank's output and LSE.
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -900,7 +907,7 @@ def extra_measurements(pa, device, peaks):
         ms, tf = fp8_timing(pa, workloads.get(name), steps=steps, warmup=2, device=device)
         out[name + "_fp8"] = {"fwd_ms_per_launch": ms, "fwd_tflops": tf,
                               "frac_of_fp8_peak": tf / (2.0 * peaks["bf16_tflops"]),
-                              "peak_basis": "2 x measured bf16 burst (nominal e4m3/bf16 ratio)"}
+                              "peak_basis": "2 x " + _basis(peaks) + " (nominal e4m3/bf16 ratio)"}
     # e4m3 quantisation (pa_quantize_e4m3) of a HunyuanVideo-sized Q tensor
     # (0.73 GB bf16, far above L2): algorithmic bytes = 2 read + 1 written per
     # element (the kernel streams x twice: amax, then convert).
