@@ -192,22 +192,32 @@ __device__ __noinline__ void store_o_rows(uint32_t tO, uint32_t stg, __nv_bfloat
   }
 }
 
-// Load this thread's fp32 row of a running state into TMEM columns
-// [tO, tO + D) (zeros where `have` is false); waits for the TMEM stores.
+// Load this thread's row of a running state: its LSE (returned; -inf for
+// rows r >= rows_left) and its fp32 O into TMEM columns [tO, tO + D) (zeros
+// where the LSE is -inf); waits for the TMEM stores.  All of the warp's
+// global loads are issued before any is used (one round trip).
 template <int D>
-__device__ __noinline__ void load_state_rows(uint32_t tO, uint32_t stg, const float* src0, int rows_left, bool have) {
+__device__ __noinline__ float load_state_rows(uint32_t tO, uint32_t stg, const float* src0, const float* lse_row,
+                                              int rows_left) {
   const int lane = threadIdx.x % 32;
   const int r0 = lane >> 3, c = lane & 7;
-#pragma unroll 1
+  const float lse0 = (lane < rows_left) ? *lse_row : -INFINITY;
+  uint4 buf[D / 32][8];
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    const uint4* src = reinterpret_cast<const uint4*>(src0 + r0 * D + ch * 32) + c;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      buf[ch][k] = (4 * k + r0 < rows_left) ? __ldg(src + k * 4 * (D / 4)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  const bool have = lse0 > -INFINITY;
+#pragma unroll
   for (int ch = 0; ch < D / 32; ++ch) {
     __syncwarp();  // the previous piece has left the staging area
-    const uint4* src = reinterpret_cast<const uint4*>(src0 + r0 * D + ch * 32) + c;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int r = 4 * k + r0;
-      uint4 x = make_uint4(0u, 0u, 0u, 0u);
-      if (r < rows_left) x = __ldg(src + k * 4 * (D / 4));
-      st_shared_v4(stg + r * 128 + ((c ^ (r & 7)) << 4), x.x, x.y, x.z, x.w);
+      st_shared_v4(stg + r * 128 + ((c ^ (r & 7)) << 4), buf[ch][k].x, buf[ch][k].y, buf[ch][k].z, buf[ch][k].w);
     }
     __syncwarp();
 #pragma unroll
@@ -225,6 +235,7 @@ __device__ __noinline__ void load_state_rows(uint32_t tO, uint32_t stg, const fl
     }
   }
   tmem_st_wait();
+  return lse0;
 }
 
 template <int D, bool kFp8 = false, bool kAcc = false>
@@ -540,13 +551,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (o_loaded) {
         const int row0 = row_of(item) - lane;  // first row of this warp's 32
         const size_t idx0 = index_of(item) - lane;
-        const float lse0 = (row0 + lane < p.Nq) ? p.acc_lse[idx0 + lane] : -INFINITY;
-        const bool have = lse0 > -INFINITY;
-        if (have) {
+        const float lse0 = load_state_rows<D>(tO, base + L::kStageOff + warp * L::kStageWarpBytes,
+                                              p.acc_o + idx0 * D, p.acc_lse + idx0 + lane, p.Nq - row0);
+        if (lse0 > -INFINITY) {
           m_ref = lse0 * 1.4426950408889634f;
           l = 1.f;
         }
-        load_state_rows<D>(tO, base + L::kStageOff + warp * L::kStageWarpBytes, p.acc_o + idx0 * D, p.Nq - row0, have);
       }
 
       for (int j = 0; j < n; ++j, ++g) {
