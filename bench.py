@@ -55,10 +55,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of the same sequence shape scaled to 24 heads (every head's items
 # are alike, so traffic grows in proportion to heads).  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "27869241fc8cb349bf30173a3896eeb6bae6e7fa39a278c5d26f738e22be35e3",
+    "source_sha256": "0107d2a56289e485af59adedd6dd9b7f1fa42c07a2b195f075fa579a6c834382",
     "bytes_per_launch": {
-        "hunyuan": (1007819520 + 124523264) * 24 // 4,
-        "flux": 85010432 + 5947648,
+        "hunyuan": (1002606592 + 123779840) * 24 // 4,
+        "flux": 85007104 + 6790400,
     },
     "capture": {
         "hunyuan": "ncu --set full, bench.py --heads 4 --steps 3 --warmup 3 --no-extra --no-cpu-baseline, x 24/4",
