@@ -556,8 +556,9 @@ def run_ours(args):
     peaks = _peaks()
     sampler = ClockSampler(local)
     fp8 = bool(getattr(args, "fp8", False))
-    if ws > 1 and args.parallel in ("ring", "ulysses"):
-        return run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=(args.parallel == "ulysses"))
+    if ws > 1 and args.parallel in ("ring", "ulysses", "usp"):
+        return run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=(args.parallel == "ulysses"),
+                        usp_degree=(args.ulysses_degree if args.parallel == "usp" else 0))
     res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier, fp8=fp8)
     if res["status"] != 0:
         raise SystemExit(f"device status {res['status']} after the timed region")
@@ -627,13 +628,14 @@ def shard_sizes(n: int, world: int):
     return [n // world + (1 if r < n % world else 0) for r in range(world)]
 
 
-def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False):
+def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_degree=0):
     """Context parallelism over the process group: rank r holds shard r of
     the query rows and of the K/V rows of workload `w` and runs
     context_parallel.ring_attention (or, with ``ulysses``, the all-to-all
-    form, which needs equal shards and heads divisible by the rank count).
-    Value = the whole problem's FLOPs per step over the slowest rank's time
-    (strong scaling)."""
+    form, which needs equal shards and heads divisible by the rank count; or,
+    with ``usp_degree`` U > 0, the Ulysses x ring grid of usp_attention, which
+    needs equal shards and heads divisible by U).  Value = the whole
+    problem's FLOPs per step over the slowest rank's time (strong scaling)."""
     import dataclasses
 
     import torch
@@ -644,6 +646,11 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False):
     nq_all, nk_all = shard_sizes(w.Nq, ws), shard_sizes(w.Nk, ws)
     if ulysses and (len(set(nq_all)) > 1 or nq_all != nk_all or w.H % ws):
         raise SystemExit(f"--parallel ulysses needs Nq = Nk divisible by {ws} and heads divisible by {ws}")
+    if usp_degree and (len(set(nq_all)) > 1 or nq_all != nk_all or w.H % usp_degree or ws % usp_degree):
+        raise SystemExit(f"--parallel usp needs Nq = Nk divisible by {ws}, and heads and {ws} ranks divisible by "
+                         f"the Ulysses degree {usp_degree}")
+    groups = cp.usp_groups(usp_degree) if usp_degree else None
+    ring_len = ws // usp_degree if usp_degree else ws
     wr = dataclasses.replace(w, Nq=nq_all[rank], Nk=nk_all[rank], chunks=(nk_all[rank],), seed=w.seed + 100 * rank)
     q, k, v = workloads.make_case(wr, device=device)
     out = torch.empty_like(q)
@@ -664,6 +671,9 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False):
     def step(timed=False):
         if ulysses:
             return cp.ulysses_attention(q, k, v, scale=w.scale, attend_full=attend_full_timed if timed else None)
+        if usp_degree:
+            return cp.usp_attention(q, k, v, groups[0], groups[1], scale=w.scale, comm_stream=comm,
+                                    attend=attend_timed if timed else None)
         return cp.ring_attention(q, k, v, kv_lens=nk_all, scale=w.scale, out=out, comm_stream=comm,
                                  attend=attend_timed if timed else None)
 
@@ -691,8 +701,9 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False):
     fl_rank = workloads.flops(w.B, w.H, nq_all[rank], w.Nk, w.d)
     launch_ms = statistics.fmean(fwd_ms)
     # ring: one fold launch per block, 1/ws of the rank's FLOPs each; Ulysses:
-    # one launch over the rank's heads and the whole sequence
-    achieved = (fl_rank / ws if not ulysses else fl_rank) / (launch_ms * 1e-3) / 1e12
+    # one launch over the rank's heads and the whole sequence; USP: one fold
+    # per ring step, 1/ring_len of the rank's FLOPs each
+    achieved = (fl_rank / ring_len if not ulysses else fl_rank) / (launch_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": None,
@@ -728,11 +739,13 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False):
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(_config(w, parallelism=(f"Ulysses attention over {ws} ranks (two NCCL all-to-alls)" if ulysses
+                                                   else f"USP over {ws} ranks: Ulysses degree {usp_degree} x ring "
+                                                        f"degree {ring_len}" if usp_degree
                                                    else f"ring attention over {ws} ranks (NCCL P2P on a second stream)")),
                            q_shards=nq_all, kv_shards=nk_all,
                            l2="each rank's K/V blocks rotate through the ring; inputs far larger than L2"),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak, "roofline": roof, "clocks": sampler.summary(),
-            "gpu_launches": args.steps * (1 if ulysses else ws),
+            "gpu_launches": args.steps * (1 if ulysses else ring_len),
             "e2e": {"value": fl * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
                     "d2h_bytes_per_step": int(out.numel() * 2 + out.numel() // w.d * 4), "steps": e_steps,
@@ -949,8 +962,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="hunyuan", choices=sorted(workloads.WORKLOADS))
-    ap.add_argument("--parallel", choices=["ring", "ulysses", "replicas"], default="ring",
-                    help="with more than one GPU: ring or Ulysses attention over the ranks, or independent replicas")
+    ap.add_argument("--parallel", choices=["ring", "ulysses", "usp", "replicas"], default="ring",
+                    help="with more than one GPU: ring, Ulysses or USP (Ulysses x ring) attention over the ranks, "
+                         "or independent replicas")
+    ap.add_argument("--ulysses-degree", type=int, default=2,
+                    help="with --parallel usp: ranks per Ulysses group (the ring runs across the groups)")
     ap.add_argument("--fp8", action="store_true",
                     help="time the e4m3 forward (pa_attn_fwd_fp8) instead of bf16; one-chunk workloads")
     ap.add_argument("--heads", type=int, default=None,

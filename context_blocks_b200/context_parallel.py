@@ -19,6 +19,12 @@ Both follow the diffusers guide "Context parallelism":
   its heads with ``pa_attn_fwd``, and a second all-to-all turns the output
   back.  It needs the head count, and the per-device sequence length, to be
   the same on every device and the heads to divide by the device count.
+* section "Unified Attention" (USP): the devices form a grid of
+  ulysses_degree x ring_degree.  Within each group of ulysses_degree
+  consecutive ranks the Ulysses all-to-all turns sequence shards into head
+  shards over the group's part of the sequence; the ring then runs across
+  the groups (ranks holding the same heads), and a second all-to-all turns
+  the result back.
 
 The functions take a ``torch.distributed`` process group (NCCL for CUDA
 tensors).  The arithmetic of a step is passed in as ``attend`` /
@@ -30,7 +36,7 @@ from __future__ import annotations
 
 from typing import Callable, List, Optional, Sequence
 
-__all__ = ["ring_schedule", "ring_attention", "ulysses_attention"]
+__all__ = ["ring_schedule", "ring_attention", "ulysses_attention", "usp_groups", "usp_attention"]
 
 
 def ring_schedule(rank: int, world: int) -> List[dict]:
@@ -90,8 +96,11 @@ def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
         raise ValueError(f"kv_lens {kv_lens} does not match the group ({world} ranks, own block {k.shape[2]})")
 
     cuda = q.is_cuda
-    o_acc = torch.empty((B, H, n_q, d), dtype=torch.float32, device=q.device)
-    lse_acc = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
+    # The running state is fp32 for the library's kernels; CPU tensors (the
+    # exchange tests) keep at least their own precision.
+    state_dtype = torch.float32 if cuda else torch.promote_types(q.dtype, torch.float32)
+    o_acc = torch.empty((B, H, n_q, d), dtype=state_dtype, device=q.device)
+    lse_acc = torch.empty((B, H, n_q), dtype=state_dtype, device=q.device)
     if out is None:
         out = torch.empty_like(q)
     if world == 1:
@@ -170,6 +179,31 @@ def _a2a(x, group):
     return y
 
 
+def _seq_to_heads(x, group):
+    """[B, H, n, ...] sequence shard -> [B, H/P, P*n, ...]: head group j goes to
+    rank j of `group`, and the P shards of the group's ranks line up along
+    the sequence in rank order."""
+    import torch.distributed as dist
+    P = dist.get_world_size(group)
+    B, H, n = x.shape[:3]
+    rest = tuple(x.shape[3:])
+    xs = x.reshape(B, P, H // P, n, *rest).transpose(0, 1).contiguous()
+    y = _a2a(xs, group)                                      # [P(src rank), B, H/P, n, ...]
+    return y.permute(1, 2, 0, *range(3, y.dim())).reshape(B, H // P, P * n, *rest).contiguous()
+
+
+def _heads_to_seq(y, group):
+    """The inverse of _seq_to_heads: [B, H/P, P*n, ...] -> [B, H, n, ...]."""
+    import torch.distributed as dist
+    P = dist.get_world_size(group)
+    B, Hp, Pn = y.shape[:3]
+    n = Pn // P
+    rest = tuple(y.shape[3:])
+    ys = y.reshape(B, Hp, P, n, *rest).permute(2, 0, 1, *range(3, y.dim() + 1)).contiguous()
+    z = _a2a(ys, group)                                      # [P(src head group), B, H/P, n, ...]
+    return z.transpose(0, 1).reshape(B, Hp * P, n, *rest).contiguous()
+
+
 def _default_attend_full(q, k, v, scale):
     from ._binding import attn_fwd
     return attn_fwd(q, k, v, scale=scale)
@@ -181,7 +215,6 @@ def ulysses_attention(q, k, v, group=None, scale: Optional[float] = None, attend
     rank's shard of the output (o [B,H,n,d], lse [B,H,n] fp32) out."""
     import math
 
-    import torch
     import torch.distributed as dist
 
     P = dist.get_world_size(group)
@@ -193,20 +226,63 @@ def ulysses_attention(q, k, v, group=None, scale: Optional[float] = None, attend
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     attend_full = attend_full or _default_attend_full
-    Hp = H // P
-
-    def to_heads(x):
-        # [B, H, n, d] -> send head group j to rank j -> [B, Hp, P*n, d] (sequence in rank order)
-        xs = x.reshape(B, P, Hp, n, *x.shape[3:]).transpose(0, 1).contiguous()
-        y = _a2a(xs, group)                                      # [P(src rank), B, Hp, n, ...]
-        return y.permute(1, 2, 0, *range(3, y.dim())).reshape(B, Hp, P * n, *x.shape[3:]).contiguous()
-
-    def to_seq(y):
-        # [B, Hp, P*n, ...] -> back to [B, H, n, ...] for this rank's sequence shard
-        ys = y.reshape(B, Hp, P, n, *y.shape[3:]).permute(2, 0, 1, *range(3, y.dim() + 1)).contiguous()
-        z = _a2a(ys, group)                                      # [P(src head group), B, Hp, n, ...]
-        return z.transpose(0, 1).reshape(B, H, n, *y.shape[3:]).contiguous()
-
-    qh, kh, vh = to_heads(q), to_heads(k), to_heads(v)
+    qh, kh, vh = _seq_to_heads(q, group), _seq_to_heads(k, group), _seq_to_heads(v, group)
     o_h, lse_h = attend_full(qh, kh, vh, scale)
-    return to_seq(o_h), to_seq(lse_h)
+    return _heads_to_seq(o_h, group), _heads_to_seq(lse_h, group)
+
+
+def usp_groups(ulysses_degree: int, group=None):
+    """The process groups of a ulysses_degree x ring_degree grid over `group`
+    (default: the whole world; its size must divide by ulysses_degree).
+    Returns (ulysses_group, ring_group) of the calling rank.  Group rank r
+    has Ulysses index r % ulysses_degree and ring index r // ulysses_degree:
+    a Ulysses group is ulysses_degree consecutive ranks, a ring group the
+    ranks with the same Ulysses index.  Every rank of `group` must call this
+    (the groups are created collectively, in the same order everywhere)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    U = int(ulysses_degree)
+    if U < 1 or world % U:
+        raise ValueError(f"ulysses_degree {U} does not divide {world} ranks")
+    R = world // U
+    glob = (lambda r: r) if group is None else (lambda r: dist.get_global_rank(group, r))
+    mine_u = mine_r = None
+    for g in range(R):
+        ranks = [glob(g * U + u) for u in range(U)]
+        pg = dist.new_group(ranks)
+        if rank // U == g:
+            mine_u = pg
+    for u in range(U):
+        ranks = [glob(g * U + u) for g in range(R)]
+        pg = dist.new_group(ranks)
+        if rank % U == u:
+            mine_r = pg
+    return mine_u, mine_r
+
+
+def usp_attention(q, k, v, ulysses_group, ring_group, scale: Optional[float] = None, attend: Optional[Callable] = None,
+                  comm_stream=None, trace: Optional[list] = None):
+    """Unified (Ulysses x ring) attention of this rank's sequence shard q, k, v
+    [B,H,n,d] (the same n and H on every rank; H divisible by the Ulysses
+    degree) over the whole sequence, which is sharded over the ranks in
+    group-rank order (see usp_groups).  Returns (o [B,H,n,d], lse [B,H,n]).
+    ``attend`` is the fold step passed to ring_attention."""
+    import math
+
+    import torch.distributed as dist
+
+    U = dist.get_world_size(ulysses_group)
+    R = dist.get_world_size(ring_group)
+    B, H, n, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("USP needs q, k, v of one shape [B,H,n,d] on every rank")
+    if H % U:
+        raise ValueError(f"{H} heads do not divide over a Ulysses degree of {U}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    qh, kh, vh = (_seq_to_heads(t, ulysses_group) for t in (q, k, v))   # [B, H/U, U*n, d]
+    out = qh.new_empty(qh.shape)
+    o_h, lse_h = ring_attention(qh, kh, vh, group=ring_group, kv_lens=[U * n] * R, scale=scale, out=out,
+                                attend=attend, comm_stream=comm_stream, trace=trace)
+    return _heads_to_seq(o_h, ulysses_group), _heads_to_seq(lse_h, ulysses_group)

@@ -195,3 +195,38 @@ def test_ulysses_attention_gloo(world, H):
         err_o, err_l, seen = got[rank]
         assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
         assert seen == [(2, H // world, n * world, 8)]     # its heads, the whole sequence
+
+
+def _usp_rank(rank, world, port, U, n, H, out_q):
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import usp_attention, usp_groups
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        ug, rg = usp_groups(U)
+        q, k, v = _global_case(9, 2, H, n * world, 8)
+        sl = slice(rank * n, (rank + 1) * n)
+        trace = []
+        o, lse = usp_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
+                               ug, rg, scale=SCALE, attend=_oracle_fold, trace=trace)
+        o_ref, l_ref = oracle.attention(q[:, :, sl], k, v, SCALE)
+        out_q.put((rank, float(np.abs(o.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()),
+                   [t["block"] for t in trace], dist.get_world_size(ug), dist.get_world_size(rg)))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("U", [1, 2, 4])
+def test_usp_attention_gloo(U):
+    """diffusers "Context parallelism", section "Unified Attention": 4 ranks
+    as a Ulysses x ring grid (4 x 1, 2 x 2, 1 x 4); every rank gets the
+    attention of its queries over the whole sequence."""
+    world, n, H = 4, 3, 4
+    got = _run(_usp_rank, world, U, n, H)
+    R = world // U
+    for rank in range(world):
+        err_o, err_l, blocks, u_size, r_size = got[rank]
+        assert err_o < 1e-12 and err_l < 1e-12, (U, rank, err_o, err_l)
+        assert (u_size, r_size) == (U, R)
+        g = rank // U
+        assert blocks == [(g - s) % R for s in range(R)]     # the ring runs across the groups
