@@ -207,16 +207,22 @@ def aggregate_throughput(flops_per_step_per_rank: float, steps: int, world: int,
 # ------------------------------------------------------------------ our arm
 
 class Step:
-    """Buffers and launches of one hot-path step on one workload."""
+    """Buffers and launches of one hot-path step on one workload.  A chunked
+    workload runs in `mode`: ``chunks`` (pa_attn_fwd per chunk, then
+    pa_attn_merge), ``fused`` (one pa_attn_fwd_chunks launch) or ``fold``
+    (pa_attn_fwd_accum per chunk into an fp32 running state)."""
 
-    def __init__(self, w: workloads.Workload, sets: int, device, fp8: bool = False, pa=None):
+    def __init__(self, w: workloads.Workload, sets: int, device, fp8: bool = False, pa=None, mode: str = "chunks"):
         import torch
         self.w = w
         self.fp8 = fp8
+        self.mode = mode
         self.sets = []
         n = len(w.chunks)
         if fp8 and n != 1:
             raise SystemExit("--fp8 times the single-chunk e4m3 forward: pick a one-chunk workload")
+        if mode == "fused" and n > 8:
+            raise SystemExit("--mode fused takes at most 8 chunks")
         for s in range(sets):
             q, k, v = workloads.make_case(w, device=device, seed=w.seed + 1000 * s)
             if fp8:
@@ -233,11 +239,13 @@ class Step:
             o = torch.empty_like(q)
             lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
             o_parts = lse_parts = None
-            if n > 1:
+            if n > 1 and mode == "chunks":
                 o_parts = torch.empty((n,) + tuple(q.shape), dtype=torch.bfloat16, device=device)
                 lse_parts = torch.empty((n,) + tuple(q.shape[:3]), dtype=torch.float32, device=device)
+            if mode == "fold":  # the fp32 running state (O; LSE goes to `lse`)
+                o_parts = torch.empty(q.shape, dtype=torch.float32, device=device)
             self.sets.append((q, pairs, o, lse, o_parts, lse_parts))
-        self.launches_per_step = n + (1 if n > 1 else 0)
+        self.launches_per_step = {"chunks": n + (1 if n > 1 else 0), "fused": 1, "fold": n}[mode]
 
     def bytes_resident(self) -> int:
         tot = 0
@@ -248,7 +256,7 @@ class Step:
         for q, pairs, o, lse, op, lp in self.sets:
             tot += q.numel() * 2 + sum(k.numel() * 4 for k, _ in pairs) + o.numel() * 2 + lse.numel() * 4
             if op is not None:
-                tot += op.numel() * 2 + lp.numel() * 4
+                tot += op.numel() * op.element_size() + (lp.numel() * 4 if lp is not None else 0)
         return tot
 
     def run(self, i: int, pa, fwd_events=None, merge_events=None):
@@ -262,6 +270,22 @@ class Step:
             return
         q, pairs, o, lse, o_parts, lse_parts = self.sets[i % len(self.sets)]
         n = len(pairs)
+        if self.mode == "fused":
+            if fwd_events is not None:
+                fwd_events[0].append(_record())
+            pa.attn_fwd_chunks(q, [k for k, _ in pairs], [v for _, v in pairs], scale=self.w.scale, out=o, lse=lse)
+            if fwd_events is not None:
+                fwd_events[1].append(_record())
+            return
+        if self.mode == "fold":
+            for p, (k, v) in enumerate(pairs):
+                if fwd_events is not None:
+                    fwd_events[0].append(_record())
+                pa.attn_fwd_accum(q, k, v, o_parts, lse, first=(p == 0), final=(p == n - 1),
+                                  out=o if p == n - 1 else None, scale=self.w.scale)
+                if fwd_events is not None:
+                    fwd_events[1].append(_record())
+            return
         for p, (k, v) in enumerate(pairs):
             out = o if n == 1 else o_parts[p]
             ls = lse if n == 1 else lse_parts[p]
@@ -303,11 +327,11 @@ def _sets_for(w: workloads.Workload, fp8: bool = False) -> int:
     return max(1, min(8, math.ceil(2.5 * L2_BYTES / per_set)))
 
 
-def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, fp8=False):
+def time_workload(pa, w, steps, warmup, device, sampler=None, barrier=None, fp8=False, mode="chunks"):
     """Device time of `steps` steps (CUDA events on the launching stream,
     synchronised on both sides).  Returns a dict of timings."""
     import torch
-    st = Step(w, _sets_for(w, fp8), device, fp8=fp8, pa=pa)
+    st = Step(w, _sets_for(w, fp8), device, fp8=fp8, pa=pa, mode=mode)
     for i in range(warmup):
         st.run(i, pa)
     torch.cuda.synchronize()
@@ -559,7 +583,8 @@ def run_ours(args):
     if ws > 1 and args.parallel in ("ring", "ulysses", "usp"):
         return run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=(args.parallel == "ulysses"),
                         usp_degree=(args.ulysses_degree if args.parallel == "usp" else 0))
-    res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier, fp8=fp8)
+    mode = args.mode if len(w.chunks) > 1 else "chunks"
+    res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier, fp8=fp8, mode=mode)
     if res["status"] != 0:
         raise SystemExit(f"device status {res['status']} after the timed region")
     max_ms = max_over_ranks(res["total_ms"], device)
@@ -569,7 +594,7 @@ def run_ours(args):
     # Roofline of the dominant kernel (attn_fwd): algorithmic FLOPs per launch
     # over its mean launch duration, against the measured bf16 dense peak.
     fwd_mean_ms = statistics.fmean(res["fwd_ms"])
-    fl_launch = fl / len(w.chunks)
+    fl_launch = fl if mode == "fused" else fl / len(w.chunks)
     achieved = fl_launch / (fwd_mean_ms * 1e-3) / 1e12
     traffic = None
     if (not fp8 and len(w.chunks) == 1 and w.name in NCU_TRAFFIC["bytes_per_launch"]
@@ -577,12 +602,16 @@ def run_ours(args):
         traffic = NCU_TRAFFIC["bytes_per_launch"][w.name]
     # e4m3 contractions: the measured bf16 peak times the nominal e4m3/bf16 ratio of 2
     peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
-    alg_bytes = workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk // len(w.chunks), w.d)
+    alg_bytes = workloads.fwd_bytes(w.B, w.H, w.Nq, w.Nk if mode == "fused" else w.Nk // len(w.chunks), w.d)
+    if mode == "fold":  # the fp32 running state read and written
+        alg_bytes += 8 * w.B * w.H * w.Nq * w.d
     if fp8:
         alg_bytes -= (w.Nq + 2 * (w.Nk // len(w.chunks))) * w.d * w.B * w.H
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic,
-            "kernel": f"attn_fwd_kernel<{w.d}, {'true' if fp8 else 'false'}, false>", "launch_ms": fwd_mean_ms,
+            "kernel": (f"attn_fwd_kernel<{w.d}, {'true' if fp8 else 'false'}, {'true' if mode == 'fold' else 'false'}>"
+                       + {"chunks": "", "fused": f" over a table of {len(w.chunks)} chunks",
+                          "fold": " (accumulate mode)"}[mode]), "launch_ms": fwd_mean_ms,
             "peak_basis": (_basis(peaks)
                            + (" x 2, the nominal e4m3/bf16 ratio" if fp8 else "")
                            + f"; frac of sustained {achieved / (peak * peaks['bf16_tflops_sustained'] / peaks['bf16_tflops']):.3f}"),
@@ -591,8 +620,8 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
-            "config": _config(w, res["sets"], res["resident_mb"], "replicas (one independent step per GPU)"
-                              if ws > 1 else "one GPU"),
+            "config": dict(_config(w, res["sets"], res["resident_mb"], "replicas (one independent step per GPU)"
+                                   if ws > 1 else "one GPU"), mode=mode),
             ("pct_of_e4m3_peak" if fp8 else "pct_of_bf16_peak"): 100.0 * (value / ws) / peak,
             "roofline": roof, "clocks": sampler.summary(), "gpu_launches": res["launches"]}
     if res["merge_ms"]:
@@ -967,6 +996,9 @@ def main(argv=None):
                          "or independent replicas")
     ap.add_argument("--ulysses-degree", type=int, default=2,
                     help="with --parallel usp: ranks per Ulysses group (the ring runs across the groups)")
+    ap.add_argument("--mode", choices=["chunks", "fused", "fold"], default="chunks",
+                    help="how a chunked workload's step runs: pa_attn_fwd per chunk + pa_attn_merge, one "
+                         "pa_attn_fwd_chunks launch, or pa_attn_fwd_accum folds")
     ap.add_argument("--fp8", action="store_true",
                     help="time the e4m3 forward (pa_attn_fwd_fp8) instead of bf16; one-chunk workloads")
     ap.add_argument("--heads", type=int, default=None,
