@@ -371,7 +371,7 @@ class _Null:
         return False
 
 
-def e2e_throughput(pa, w, steps, device, fp8: bool = False):
+def e2e_throughput(pa, w, steps, device, fp8: bool = False, mode: str = "chunks"):
     """Same metric through the public API from pinned HOST buffers: every
     step copies q and the K/V chunks host->device, runs the step, and copies
     o and lse device->host; all inside the timed region.
@@ -381,7 +381,8 @@ def e2e_throughput(pa, w, steps, device, fp8: bool = False):
     step's attention and device->host copy (the copy engines of the two
     directions and the SMs work at the same time).  Each step still moves
     all of its own bytes.  With fp8 the host holds e4m3 codes (quantised once
-    by the library, scales kept on the device) and each step uploads those."""
+    by the library, scales kept on the device) and each step uploads those.
+    A chunked workload runs in `mode`, as the device-timed step does."""
     import torch
     q, k, v = workloads.make_case(w, device=device)
     B, H, Nq, d = q.shape
@@ -401,8 +402,11 @@ def e2e_throughput(pa, w, steps, device, fp8: bool = False):
         def __init__(self):
             self.stream = torch.cuda.Stream(device=device)
             self.dev_in = [torch.empty(h.shape, dtype=h.dtype, device=device) for h in host_in]
-            self.o_parts = torch.empty((n, B, H, Nq, d), dtype=torch.bfloat16, device=device) if n > 1 else None
-            self.lse_parts = torch.empty((n, B, H, Nq), dtype=torch.float32, device=device) if n > 1 else None
+            self.o_parts = (torch.empty((n, B, H, Nq, d), dtype=torch.bfloat16, device=device)
+                            if n > 1 and mode == "chunks" else None)
+            self.lse_parts = (torch.empty((n, B, H, Nq), dtype=torch.float32, device=device)
+                              if n > 1 and mode == "chunks" else None)
+            self.o_acc = torch.empty((B, H, Nq, d), dtype=torch.float32, device=device) if mode == "fold" else None
             self.o = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=device)
             self.lse = torch.empty((B, H, Nq), dtype=torch.float32, device=device)
             self.ho = torch.empty(self.o.shape, dtype=self.o.dtype, pin_memory=True)
@@ -418,8 +422,18 @@ def e2e_throughput(pa, w, steps, device, fp8: bool = False):
                                     stream=self.stream)
                 else:
                     dq, rest = self.dev_in[0], self.dev_in[1:]
-                    pa.blockwise_attention(dq, rest[0::2], rest[1::2], scale=w.scale, o_parts=self.o_parts,
-                                           lse_parts=self.lse_parts, out=self.o, lse=self.lse, stream=self.stream)
+                    ks, vs = rest[0::2], rest[1::2]
+                    if mode == "fused":
+                        pa.attn_fwd_chunks(dq, ks, vs, scale=w.scale, out=self.o, lse=self.lse, stream=self.stream)
+                    elif mode == "fold":
+                        for c in range(n):
+                            pa.attn_fwd_accum(dq, ks[c], vs[c], self.o_acc, self.lse, first=(c == 0),
+                                              final=(c == n - 1), out=self.o if c == n - 1 else None,
+                                              scale=w.scale, stream=self.stream)
+                    else:
+                        pa.blockwise_attention(dq, ks, vs, scale=w.scale, o_parts=self.o_parts,
+                                               lse_parts=self.lse_parts, out=self.o, lse=self.lse,
+                                               stream=self.stream)
                 self.ho.copy_(self.o, non_blocking=True)
                 self.hl.copy_(self.lse, non_blocking=True)
 
@@ -446,7 +460,7 @@ def e2e_throughput(pa, w, steps, device, fp8: bool = False):
     fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
     return {"value": fl * steps / (ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps,
-            "pipelining": "2 streams, double-buffered device tensors"}
+            "pipelining": "2 streams, double-buffered device tensors", "mode": mode}
 
 
 # ------------------------------------------------------------ CPU (oracle) leg
@@ -631,7 +645,7 @@ def run_ours(args):
                          "peak_gbs": peaks["hbm_gbs"]}
 
     if rank == 0 or ws > 1:
-        line["e2e"] = e2e_throughput(pa, w, steps=max(3, min(args.steps, 20)), device=device, fp8=fp8)
+        line["e2e"] = e2e_throughput(pa, w, steps=max(3, min(args.steps, 20)), device=device, fp8=fp8, mode=mode)
         if ws > 1:
             line["e2e"]["value"] = max_over_ranks(-line["e2e"]["value"], device) * -1 * ws
 
