@@ -91,3 +91,35 @@ def test_random_shape(pa, i):
     torch.cuda.synchronize()
     assert pa.poll_device_status() == pa.PA_OK
     assert_close(o, lse, o_ref, l_ref, f"random no-alloc, {what}")
+
+
+def _fp8_case(i):
+    r = np.random.default_rng(9090 + i)
+    return (int(r.integers(1, 3)), int(r.integers(1, 4)), int(r.integers(1, 700)), int(r.integers(64, 1500)),
+            int(r.integers(0, 2**31)))
+
+
+@pytest.mark.parametrize("i", range(8))
+def test_random_shape_e4m3(pa, i):
+    """The e4m3 forward on random shapes, with the scales made on the device
+    by the library's quantiser (pa_attn_fwd_fp8_dev) and given on the host
+    (pa_attn_fwd_fp8): both against the oracle on the dequantised codes, with
+    the e4m3 bounds."""
+    from tests._parity import assert_close_fp8
+    B, H, Nq, Nk, seed = _fp8_case(i)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q = torch.randn((B, H, Nq, 128), generator=g, device="cuda").to(torch.bfloat16)
+    k = torch.randn((B, H, Nk, 128), generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn((B, H, Nk, 128), generator=g, device="cuda").to(torch.bfloat16)
+    (q8, sq), (k8, sk), (v8, sv) = pa.quantize_e4m3(q), pa.quantize_e4m3(k), pa.quantize_e4m3(v)
+    scale = 1.0 / math.sqrt(128)
+    o_dev, l_dev = pa.attn_fwd_fp8(q8, k8, v8, sq, sk, sv, scale=scale)
+    o_host, l_host = pa.attn_fwd_fp8(q8, k8, v8, float(sq.item()), float(sk.item()), float(sv.item()), scale=scale)
+    torch.cuda.synchronize()
+    assert pa.poll_device_status() == pa.PA_OK
+    deq = [x.cpu().double() * float(s.item()) for x, s in ((q8, sq), (k8, sk), (v8, sv))]
+    o_ref, l_ref = oracle.attention(deq[0], deq[1], deq[2], scale)
+    what = f"e4m3 B={B} H={H} Nq={Nq} Nk={Nk}"
+    v_max = float(deq[2].abs().max())
+    assert_close_fp8(o_dev, l_dev, o_ref, l_ref, v_max, f"random {what}, device scales")
+    assert_close_fp8(o_host, l_host, o_ref, l_ref, v_max, f"random {what}, host scales")
