@@ -475,7 +475,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             break;
           }
           tc_fence_after();
-          if (leader) issue_pv(i, sv, true, (kPParts - 1) * kKkPerPart, kBN / kKPerMma);
+          // The last part accumulates unless it is also the first of the item.
+          if (leader)
+            issue_pv(i, sv, kPParts > 1 || o_loaded || j > 0, (kPParts - 1) * kKkPerPart, kBN / kKPerMma);
           if (leader && i == 1) umma_commit(bar_kv_empty0 + 8 * sv);
           __syncwarp();
           if (more) {
