@@ -19,6 +19,8 @@
 //   warp  8    TMEM allocation + tcgen05.mma issue (the whole warp runs the
 //              loop in step, one elected lane issues)
 //   warp  9    TMA producer (Q once, then the K_j / V_j ring; same scheme)
+//   warps 10-11 (bf16 only) idle, completing warpgroup 2 for a register split
+//              that gives the softmax warps 208 registers
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128)        S_0 = Q_0 K_j^T   (P_0 is written back over it: bf16
 //                  pairs, or four e4m3 per column with e4m3 inputs)
@@ -86,9 +88,23 @@ struct KvChunks {
   int tile_start[kMaxChunks];  // key tiles before chunk c (unused entries: INT_MAX)
   int n_chunks;
 };
-constexpr int kFwdThreads = 320;   // 10 warps
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
+// bf16: 12 warps, warps 10 and 11 idle so that warps 8-11 form a warpgroup
+// for the register split below; e4m3: 10 warps, no split (measured slower).
+// The split: each sub-partition holds three warps of 168 registers at launch
+// (3 x 32 x 168 = 16128 of its 16384); warpgroup 2 (MMA, TMA, 2 idle) drops
+// to 88 and the two softmax warpgroups rise to 208 (32 x (88 + 2 x 208) =
+// 16128, the launch's own allocation).  The host checks that the kernel was
+// built with exactly kLaunchRegs registers before it launches one.
+template <bool kFp8>
+constexpr int fwd_threads() {
+  return kFp8 ? 320 : 384;
+}
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kControlRegs = 88;
+static_assert(kControlRegs + 2 * kSoftmaxRegs == 3 * kLaunchRegs, "register split must sum to the launch allocation");
 
 // kFp8: Q, K, V are e4m3 (one byte per element) instead of bf16.
 template <int D, bool kFp8 = false>
@@ -239,7 +255,7 @@ __device__ __noinline__ float load_state_rows(uint32_t tO, uint32_t stg, const f
 }
 
 template <int D, bool kFp8 = false, bool kAcc = false>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(fwd_threads<kFp8>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ KvChunks kv,
                     const FwdParams p) {
   using L = FwdLayout<D, kFp8>;
@@ -303,7 +319,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kTmaWarp) {
+  if (warp >= 10) {
+    if constexpr (!kFp8) setmaxnreg_dec<kControlRegs>();  // idle: completes warpgroup 2
+  } else if (warp == kTmaWarp) {
+    if constexpr (!kFp8) setmaxnreg_dec<kControlRegs>();
     // ------------------------------------------------------------ producer
     // The whole warp runs the loop in step; the elected lane issues the loads.
     const bool leader = elect_one();
@@ -370,6 +389,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
+    if constexpr (!kFp8) setmaxnreg_dec<kControlRegs>();
     // ------------------------------------------------------------ MMA issue
     // The whole warp runs the loop in step and waits on the barriers; the
     // elected lane issues every tcgen05.mma and tcgen05.commit.  Shared-memory
@@ -509,6 +529,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_wait(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
     __syncwarp();
   } else {
+    if constexpr (!kFp8) setmaxnreg_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax
     const int i = warp / 4;                    // query tile of this warpgroup
     const int t = threadIdx.x % 128;           // row within the tile = TMEM lane

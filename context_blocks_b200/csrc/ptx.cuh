@@ -258,6 +258,19 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Per-warpgroup register budget (all four warps of a warpgroup execute it):
+// dec returns registers to the CTA's pool, inc takes them from it.  An inc
+// that asks for more than the pool holds would wait for ever, so callers
+// size the split against the launch's own allocation.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 // 16-byte shared-memory store and load (addresses 16-byte aligned).
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
