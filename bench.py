@@ -55,10 +55,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of the same sequence shape scaled to 24 heads (every head's items
 # are alike, so traffic grows in proportion to heads).  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "9cdf98de61787c65971f29aef53bfb44b2b7c9aeb3ac265dc10e383114c70b8c",
+    "source_sha256": "28542e21366513431a57c99f33d9a07daaf713b99ada4713b67f3dcc1bdd29c8",
     "bytes_per_launch": {
-        "hunyuan": (952105984 + 123875328) * 24 // 4,
-        "flux": 85003520 + 6852352,
+        "hunyuan": (952058368 + 121527296) * 24 // 4,
+        "flux": 84987648 + 5940224,
     },
     "capture": {
         "hunyuan": "ncu --set full, bench.py --heads 4 --steps 3 --warmup 3 --no-extra --no-cpu-baseline, x 24/4",

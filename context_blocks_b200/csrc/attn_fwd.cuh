@@ -41,8 +41,8 @@
 // on the final fold, the bf16 output).
 //
 // With kFp8 the same kernel takes e4m3 Q, K, V (per-tensor scales folded into
-// the logit scale and the epilogue) and issues kind::f8f6f4 MMAs; 3 in 8 of
-// its exponentials are computed on the FMA pipe (exp2_poly2_x2).
+// the logit scale and the epilogue) and issues kind::f8f6f4 MMAs.  A share of
+// the exponentials (3 in 8 for e4m3, 1 in 8 for bf16) runs on the FMA pipe.
 //
 // Shared memory: Q (two tiles), a 4-slot K/V ring, a 4 KB output staging area
 // per softmax warp, then the barriers (230.6 KB with bf16 d = 128).
@@ -70,11 +70,14 @@ constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms; the wait itself stays bou
 constexpr int kPParts = 2;         // P is handed to the MMA warp in this many parts
 constexpr int kStages = 4;         // K/V ring slots (each holds one K or one V tile)
 constexpr int kMaxChunks = 8;      // K/V chunks one launch can consume
-// With e4m3 inputs the tensor pipe needs half the time of the exponentials,
-// so pairs e of each 32-key chunk whose bit is set here (3 in 8) take 2^x on
-// the FMA pipe (exp2_poly2_x2) instead of MUFU.  Measured: 1/4 and 1/2 are
-// slower than 3/8; in the bf16 path any share is slower.
+// Pairs e of each 32-key chunk whose bit is set here take 2^x on the FMA pipe
+// instead of MUFU.  With e4m3 inputs the tensor pipe needs half the time of
+// the exponentials, and 3 in 8 pairs pay (exp2_poly2_x2; 1/4 and 1/2 were
+// measured slower).  In the bf16 path, with the softmax warps at 208
+// registers, 1 in 8 pairs pays a little (exp2_poly3_x2; it draws more power,
+// so under the power cap the gain is smaller than per clock).
 constexpr uint32_t kPolyPairsFp8 = 0xA4A4u;
+constexpr uint32_t kPolyPairsBf16 = 0x0808u;
 
 // The K/V chunks of one launch: keys are the concatenation of the chunks, in
 // order; each chunk has its own tensor maps and its own (possibly ragged)
@@ -636,8 +639,8 @@ __global__ void __launch_bounds__(fwd_threads<kFp8>(), 1)
             tmem_st_x32(tO + ch * 32, orr);
           }
         }
-        // x = s * c - m_ref on packed pairs, P = 2^x on MUFU (with e4m3
-        // inputs 3 pairs in 8 on the FMA pipe instead), the row sum in four
+        // x = s * c - m_ref on packed pairs, P = 2^x on MUFU (a share of the
+        // pairs on the FMA pipe instead, see kPolyPairs*), the row sum in four
         // packed partial sums.
         const float neg_m = -m_ref;
         const uint64_t c2 = f2(c, c), nm2 = f2(neg_m, neg_m);
@@ -651,6 +654,8 @@ __global__ void __launch_bounds__(fwd_threads<kFp8>(), 1)
             float p0, p1;
             if (kFp8 && ((kPolyPairsFp8 >> e) & 1)) {
               f2_split(exp2_poly2_x2(x2), p0, p1);
+            } else if (!kFp8 && ((kPolyPairsBf16 >> e) & 1)) {
+              f2_split(exp2_poly3_x2(x2), p0, p1);
             } else {
               float x0, x1;
               f2_split(x2, x0, x1);

@@ -96,7 +96,8 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 
 
 // 2^x on the FMA pipe for both halves of a pair, to take load off the MUFU
-// unit in the e4m3 path (whose P is rounded to e4m3 right after).  Cody-Waite
+// unit: degree 2 in the e4m3 path (whose P is rounded to e4m3 right after),
+// degree 3 in the bf16 path (P rounded to bf16, half step 2^-9).  Cody-Waite
 // range reduction x = n + f, n = round-to-nearest(x) by adding and subtracting
 // 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by a degree-2 polynomial minimax in
 // relative error (1.73e-3; coefficients from gen_exp2_poly.py); 2^n by adding
@@ -121,6 +122,30 @@ __device__ __forceinline__ uint64_t exp2_poly2_x2(uint64_t x) {
   f2_split(p, p0, p1);
   f2_split(t, t0, t1);
   // the low bits of t hold n; shifted by 23 they land in the exponent field
+  return f2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+            __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// The same with a degree-3 polynomial (relative error 7.5e-5 on the reduced
+// range, 1.4e-4 with the float32 steps; coefficients from gen_exp2_poly.py).
+constexpr float kExp2P3C0 = 9.999280572e-01f;
+constexpr float kExp2P3C1 = 6.932609677e-01f;
+constexpr float kExp2P3C2 = 2.426111251e-01f;
+constexpr float kExp2P3C3 = 5.517166853e-02f;
+
+__device__ __forceinline__ uint64_t exp2_poly3_x2(uint64_t x) {
+  float a, b;
+  f2_split(x, a, b);
+  const uint64_t xc = f2(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const uint64_t t = f2_add(xc, f2(kRoundMagic, kRoundMagic));   // magic + n
+  const uint64_t n = f2_add(t, f2(-kRoundMagic, -kRoundMagic));  // n (exact)
+  const uint64_t fr = f2_fma(n, f2(-1.f, -1.f), xc);             // f = x - n (exact)
+  uint64_t p = f2_fma(f2(kExp2P3C3, kExp2P3C3), fr, f2(kExp2P3C2, kExp2P3C2));
+  p = f2_fma(p, fr, f2(kExp2P3C1, kExp2P3C1));
+  p = f2_fma(p, fr, f2(kExp2P3C0, kExp2P3C0));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
   return f2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
             __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }

@@ -1,4 +1,5 @@
-"""Fit the polynomial of the e4m3 kernel's FMA-pipe exponential (``exp2_poly2_x2``).
+"""Fit the polynomials of the kernels' FMA-pipe exponentials (``exp2_poly2_x2``
+for the e4m3 path, ``exp2_poly3_x2`` for the bf16 path).
 
 2^x is split as 2^n * 2^f with n = round-to-nearest(x) and f = x - n in
 [-1/2, 1/2] (Cody-Waite range reduction: W. J. Cody and W. Waite, "Software
@@ -8,11 +9,13 @@ polynomial whose coefficients minimise the maximum RELATIVE error over
 float32 exponent field.
 
 Degree 2 is enough for the e4m3 path: its P is rounded to e4m3 (relative step
-2^-4) right after, and the fit's 1.73e-3 is far below that.
+2^-4) right after, and the fit's 1.73e-3 is far below that.  The bf16 path
+rounds P to bf16 (half step 2^-9, about 2e-3) and takes degree 3 (7.5e-5).
 
-The printed coefficients are the kExp2P2C* constants of fwd_common.cuh; the
-second figure simulates the kernel's float32 steps (magic-number rounding,
-Horner steps, exponent add) against float64 exp2 over [-126, 8].
+The printed coefficients are the kExp2P2C* and kExp2P3C* constants of
+fwd_common.cuh; the second figure of each simulates the kernel's float32
+steps (magic-number rounding, Horner steps, exponent add) against float64
+exp2 over [-126, 8].
 
     python context_blocks_b200/csrc/gen_exp2_poly.py
 """
@@ -67,11 +70,12 @@ def simulate(c32: np.ndarray, x: np.ndarray) -> np.ndarray:
 
 
 if __name__ == "__main__":
-    c, e = fit()
-    c32 = c.astype(np.float32)
-    print("coefficients (c0..c2):", ", ".join(f"{v:.9e}f" for v in c32))
-    print(f"max relative error of the polynomial on [-1/2, 1/2]: {e:.3e}")
-    x = np.linspace(-126.0, 8.0, 400001)
-    r = simulate(c32, x)
-    print(f"max relative error of the float32 emulation on [-126, 8]: "
-          f"{np.max(np.abs(r - np.exp2(x)) / np.exp2(x)):.3e}")
+    for degree in (2, 3):
+        c, e = fit(degree)
+        c32 = c.astype(np.float32)
+        print(f"degree {degree} coefficients (c0..c{degree}):", ", ".join(f"{v:.9e}f" for v in c32))
+        print(f"  max relative error of the polynomial on [-1/2, 1/2]: {e:.3e}")
+        x = np.linspace(-126.0, 8.0, 400001)
+        r = simulate(c32, x)
+        print(f"  max relative error of the float32 emulation on [-126, 8]: "
+              f"{np.max(np.abs(r - np.exp2(x)) / np.exp2(x)):.3e}")
