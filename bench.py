@@ -55,10 +55,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of the same sequence shape scaled to 24 heads (every head's items
 # are alike, so traffic grows in proportion to heads).  See profiles/.
 NCU_TRAFFIC = {
-    "source_sha256": "28542e21366513431a57c99f33d9a07daaf713b99ada4713b67f3dcc1bdd29c8",
+    "source_sha256": "4f469c18af13c656294c5af86d9ef3facfc6f018fbf1d7c157a1d0fd32d30cbc",
     "bytes_per_launch": {
-        "hunyuan": (952058368 + 121527296) * 24 // 4,
-        "flux": 84987648 + 5940224,
+        "hunyuan": (967502080 + 120467712) * 24 // 4,
+        "flux": 84987904 + 5317632,
     },
     "capture": {
         "hunyuan": "ncu --set full, bench.py --heads 4 --steps 3 --warmup 3 --no-extra --no-cpu-baseline, x 24/4",
@@ -959,8 +959,10 @@ def extra_measurements(pa, device, peaks):
         out[f"hunyuan_8chunks_{mode}"] = mode_timing(pa, w8, mode, 2, 1, device)
     # The e4m3 forward on the FLUX and HunyuanVideo shapes; its peak is the
     # measured bf16 burst figure times the nominal fp8/bf16 ratio of 2.
-    for name, steps in (("flux", 20), ("hunyuan", 2)):
-        ms, tf = fp8_timing(pa, workloads.get(name), steps=steps, warmup=2, device=device)
+    # 200 FLUX launches (≈ 40 ms), like the bf16 FLUX line: a few milliseconds
+    # of launches only show the clock state the previous phase left behind.
+    for name, steps, warm in (("flux", 200, 10), ("hunyuan", 2, 2)):
+        ms, tf = fp8_timing(pa, workloads.get(name), steps=steps, warmup=warm, device=device)
         out[name + "_fp8"] = {"fwd_ms_per_launch": ms, "fwd_tflops": tf,
                               "frac_of_fp8_peak": tf / (2.0 * peaks["bf16_tflops"]),
                               "peak_basis": "2 x " + _basis(peaks) + " (nominal e4m3/bf16 ratio)"}

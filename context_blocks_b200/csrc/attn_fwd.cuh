@@ -42,7 +42,7 @@
 //
 // With kFp8 the same kernel takes e4m3 Q, K, V (per-tensor scales folded into
 // the logit scale and the epilogue) and issues kind::f8f6f4 MMAs.  A share of
-// the exponentials (3 in 8 for e4m3, 1 in 8 for bf16) runs on the FMA pipe.
+// the exponentials (1 in 4 in both paths) runs on the FMA pipe.
 //
 // Shared memory: Q (two tiles), a 4-slot K/V ring, a 4 KB output staging area
 // per softmax warp, then the barriers (230.6 KB with bf16 d = 128).
@@ -71,13 +71,13 @@ constexpr int kPParts = 2;         // P is handed to the MMA warp in this many p
 constexpr int kStages = 4;         // K/V ring slots (each holds one K or one V tile)
 constexpr int kMaxChunks = 8;      // K/V chunks one launch can consume
 // Pairs e of each 32-key chunk whose bit is set here take 2^x on the FMA pipe
-// instead of MUFU.  With e4m3 inputs the tensor pipe needs half the time of
-// the exponentials, and 3 in 8 pairs pay (exp2_poly2_x2; 1/4 and 1/2 were
-// measured slower).  In the bf16 path, with the softmax warps at 208
-// registers, 1 in 8 pairs pays a little (exp2_poly3_x2; it draws more power,
-// so under the power cap the gain is smaller than per clock).
-constexpr uint32_t kPolyPairsFp8 = 0xA4A4u;
-constexpr uint32_t kPolyPairsBf16 = 0x0808u;
+// instead of MUFU.  With the softmax warps at 208 registers, 1 in 4 pairs was
+// measured fastest in both paths: e4m3 (exp2_poly2_x2; the tensor pipe needs
+// half the time of the exponentials there) against 3/16, 5/16 and 1/2, bf16
+// (exp2_poly3_x2) against 1/8, 3/16, 5/16 and 3/8.  The FMA pipe draws more
+// power, so under the power cap the gain is smaller than per clock.
+constexpr uint32_t kPolyPairsFp8 = 0x8888u;
+constexpr uint32_t kPolyPairsBf16 = 0x8888u;
 
 // The K/V chunks of one launch: keys are the concatenation of the chunks, in
 // order; each chunk has its own tensor maps and its own (possibly ragged)
@@ -93,17 +93,14 @@ struct KvChunks {
 };
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
-// bf16: 12 warps, warps 10 and 11 idle so that warps 8-11 form a warpgroup
-// for the register split below; e4m3: 10 warps, no split (measured slower).
+// 12 warps, warps 10 and 11 idle so that warps 8-11 form a warpgroup for the
+// register split below (both paths; the e4m3 path gains 2% from it).
 // The split: each sub-partition holds three warps of 168 registers at launch
 // (3 x 32 x 168 = 16128 of its 16384); warpgroup 2 (MMA, TMA, 2 idle) drops
 // to 88 and the two softmax warpgroups rise to 208 (32 x (88 + 2 x 208) =
 // 16128, the launch's own allocation).  The host checks that the kernel was
 // built with exactly kLaunchRegs registers before it launches one.
-template <bool kFp8>
-constexpr int fwd_threads() {
-  return kFp8 ? 320 : 384;
-}
+constexpr int kFwdThreads = 384;
 constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 208;
 constexpr int kControlRegs = 88;
@@ -258,7 +255,7 @@ __device__ __noinline__ float load_state_rows(uint32_t tO, uint32_t stg, const f
 }
 
 template <int D, bool kFp8 = false, bool kAcc = false>
-__global__ void __launch_bounds__(fwd_threads<kFp8>(), 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ KvChunks kv,
                     const FwdParams p) {
   using L = FwdLayout<D, kFp8>;
@@ -323,9 +320,9 @@ __global__ void __launch_bounds__(fwd_threads<kFp8>(), 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 10) {
-    if constexpr (!kFp8) setmaxnreg_dec<kControlRegs>();  // idle: completes warpgroup 2
+    setmaxnreg_dec<kControlRegs>();  // idle: completes warpgroup 2
   } else if (warp == kTmaWarp) {
-    if constexpr (!kFp8) setmaxnreg_dec<kControlRegs>();
+    setmaxnreg_dec<kControlRegs>();
     // ------------------------------------------------------------ producer
     // The whole warp runs the loop in step; the elected lane issues the loads.
     const bool leader = elect_one();
@@ -392,7 +389,7 @@ __global__ void __launch_bounds__(fwd_threads<kFp8>(), 1)
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    if constexpr (!kFp8) setmaxnreg_dec<kControlRegs>();
+    setmaxnreg_dec<kControlRegs>();
     // ------------------------------------------------------------ MMA issue
     // The whole warp runs the loop in step and waits on the barriers; the
     // elected lane issues every tcgen05.mma and tcgen05.commit.  Shared-memory
@@ -532,7 +529,7 @@ __global__ void __launch_bounds__(fwd_threads<kFp8>(), 1)
     mbar_wait(bar_drain, 0, nullptr, p.status, kStatusTimeout, lim);
     __syncwarp();
   } else {
-    if constexpr (!kFp8) setmaxnreg_inc<kSoftmaxRegs>();
+    setmaxnreg_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax
     const int i = warp / 4;                    // query tile of this warpgroup
     const int t = threadIdx.x % 128;           // row within the tile = TMEM lane

@@ -222,16 +222,14 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
     if (!st->fwd_attr[slot]) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocBytes);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-      if constexpr (!kFp8) {
-        // The kernel's register split assumes this launch allocation; with
-        // any other count its setmaxnreg.inc could wait for ever.
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, kern);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-        if (fa.numRegs != pa::single::kLaunchRegs)
-          return fail(PA_ERR_UNSUPPORTED, "forward kernel built with %d registers per thread, the register split "
-                      "needs %d", fa.numRegs, pa::single::kLaunchRegs);
-      }
+      // The kernel's register split assumes this launch allocation; with any
+      // other count its setmaxnreg.inc could wait for ever.
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      if (fa.numRegs != pa::single::kLaunchRegs)
+        return fail(PA_ERR_UNSUPPORTED, "forward kernel built with %d registers per thread, the register split "
+                    "needs %d", fa.numRegs, pa::single::kLaunchRegs);
       st->fwd_attr[slot] = true;
     }
   }
@@ -259,7 +257,7 @@ int launch_fwd(DeviceState* st, const void* q, const void* const* k, const void*
   if (items > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many query blocks");
   prm.items = static_cast<int>(items);
   const unsigned grid = static_cast<unsigned>(std::min<long long>(items, st->sm_count));
-  kern<<<grid, pa::single::fwd_threads<kFp8>(), L::kAllocBytes, stream>>>(tq, kv, prm);
+  kern<<<grid, pa::single::kFwdThreads, L::kAllocBytes, stream>>>(tq, kv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd launch");
   return PA_OK;
