@@ -19,7 +19,7 @@
 //   warp  8    TMEM allocation + tcgen05.mma issue (the whole warp runs the
 //              loop in step, one elected lane issues)
 //   warp  9    TMA producer (Q once, then the K_j / V_j ring; same scheme)
-//   warps 10-11 (bf16 only) idle, completing warpgroup 2 for a register split
+//   warps 10-11 idle, completing warpgroup 2 for a register split
 //              that gives the softmax warps 208 registers
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128)        S_0 = Q_0 K_j^T   (P_0 is written back over it: bf16
