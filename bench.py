@@ -14,10 +14,12 @@ the device time.
 Multi-GPU: one process per GPU (torchrun).  By default (``--parallel ring``)
 the ranks run Ring Attention over the named workload (diffusers "Context
 parallelism", section "Ring Attention"): each rank holds 1/N of the query
-rows and of the K/V rows, folds each K/V block into its running state with
-``pa_attn_fwd_accum`` while the next block arrives from the previous rank
-over NCCL on a second stream.  The whole problem is fixed as N grows, so
-scaling is strong.  ``--parallel replicas`` runs an independent copy of the
+rows and of the K/V rows and attends to each K/V block while the next one
+arrives from the previous rank over NCCL on a second stream: with the default
+``--mode chunks`` each block's partial comes from ``pa_attn_fwd`` and one
+``pa_attn_merge`` combines them after the last block; with ``--mode fold``
+each block is folded into an fp32 running state by ``pa_attn_fwd_accum``.
+The whole problem is fixed as N grows, so scaling is strong.  ``--parallel replicas`` runs an independent copy of the
 single-GPU step on every rank instead (weak scaling, no data-path
 collective).  Either way the process group provides the barrier and the max
 over ranks of the timed region.
@@ -671,6 +673,11 @@ def shard_sizes(n: int, world: int):
     return [n // world + (1 if r < n % world else 0) for r in range(world)]
 
 
+def _ring_how(partials: bool) -> str:
+    return ("; per-block partials (pa_attn_fwd) + one pa_attn_merge" if partials
+            else "; per-block folds into an fp32 state (pa_attn_fwd_accum)")
+
+
 def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_degree=0):
     """Context parallelism over the process group: rank r holds shard r of
     the query rows and of the K/V rows of workload `w` and runs
@@ -692,6 +699,9 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
     if usp_degree and (len(set(nq_all)) > 1 or nq_all != nk_all or w.H % usp_degree or ws % usp_degree):
         raise SystemExit(f"--parallel usp needs Nq = Nk divisible by {ws}, and heads and {ws} ranks divisible by "
                          f"the Ulysses degree {usp_degree}")
+    if args.mode == "fused" and not ulysses:
+        raise SystemExit("--mode fused is a one-GPU mode: the ring's blocks arrive one at a time")
+    partials = not ulysses and args.mode == "chunks"
     groups = cp.usp_groups(usp_degree) if usp_degree else None
     ring_len = ws // usp_degree if usp_degree else ws
     wr = dataclasses.replace(w, Nq=nq_all[rank], Nk=nk_all[rank], chunks=(nk_all[rank],), seed=w.seed + 100 * rank)
@@ -705,6 +715,11 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
         pa.attn_fwd_accum(qq, kk, vv, o_acc, lse_acc, first=first, final=final, out=o, scale=scale)
         fwd_ev[1].append(_record())
 
+    def attend_part_timed(qq, kk, vv, o_part, lse_part, scale):
+        fwd_ev[0].append(_record())
+        pa.attn_fwd(qq, kk, vv, scale=scale, out=o_part, lse=lse_part)
+        fwd_ev[1].append(_record())
+
     def attend_full_timed(qq, kk, vv, scale):
         fwd_ev[0].append(_record())
         res = pa.attn_fwd(qq, kk, vv, scale=scale)
@@ -716,9 +731,11 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
             return cp.ulysses_attention(q, k, v, scale=w.scale, attend_full=attend_full_timed if timed else None)
         if usp_degree:
             return cp.usp_attention(q, k, v, groups[0], groups[1], scale=w.scale, comm_stream=comm,
-                                    attend=attend_timed if timed else None)
+                                    attend=attend_timed if timed else None, partials=partials,
+                                    attend_part=attend_part_timed if timed else None)
         return cp.ring_attention(q, k, v, kv_lens=nk_all, scale=w.scale, out=out, comm_stream=comm,
-                                 attend=attend_timed if timed else None)
+                                 attend=attend_timed if timed else None, partials=partials,
+                                 attend_part=attend_part_timed if timed else None)
 
     for _ in range(args.warmup):
         step()
@@ -740,7 +757,8 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
     fl = workloads.flops(w.B, w.H, w.Nq, w.Nk, w.d)
     value = fl * args.steps / (max_ms * 1e-3) / 1e12
     fwd_ms = [a.elapsed_time(b) for a, b in zip(*fwd_ev)]
-    # the fold kernel: this rank's FLOPs per ring pass over its launches
+    # the forward kernel (the fold, or the plain forward of a block's partial):
+    # this rank's FLOPs per ring pass over its launches
     fl_rank = workloads.flops(w.B, w.H, nq_all[rank], w.Nk, w.d)
     launch_ms = statistics.fmean(fwd_ms)
     # ring: one fold launch per block, 1/ws of the rank's FLOPs each; Ulysses:
@@ -750,7 +768,7 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
     peak = peaks["bf16_tflops"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": None,
-            "kernel": f"attn_fwd_kernel<{w.d}, false, {'false' if ulysses else 'true'}>",
+            "kernel": f"attn_fwd_kernel<{w.d}, false, {'false' if ulysses or partials else 'true'}>",
             "launch_ms": launch_ms,
             "peak_basis": f"{_basis(peaks)}, rank {rank}"}
     # End to end: each step uploads this rank's shards from pinned host
@@ -783,12 +801,13 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(_config(w, parallelism=(f"Ulysses attention over {ws} ranks (two NCCL all-to-alls)" if ulysses
                                                    else f"USP over {ws} ranks: Ulysses degree {usp_degree} x ring "
-                                                        f"degree {ring_len}" if usp_degree
-                                                   else f"ring attention over {ws} ranks (NCCL P2P on a second stream)")),
+                                                        f"degree {ring_len}" + _ring_how(partials) if usp_degree
+                                                   else f"ring attention over {ws} ranks (NCCL P2P on a second "
+                                                        f"stream)" + _ring_how(partials))),
                            q_shards=nq_all, kv_shards=nk_all,
                            l2="each rank's K/V blocks rotate through the ring; inputs far larger than L2"),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak, "roofline": roof, "clocks": sampler.summary(),
-            "gpu_launches": args.steps * (1 if ulysses else ring_len),
+            "gpu_launches": args.steps * (1 if ulysses else ring_len + (1 if partials else 0)),
             "e2e": {"value": fl * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
                     "d2h_bytes_per_step": int(out.numel() * 2 + out.numel() // w.d * 4), "steps": e_steps,
@@ -1014,7 +1033,8 @@ def main(argv=None):
                     help="with --parallel usp: ranks per Ulysses group (the ring runs across the groups)")
     ap.add_argument("--mode", choices=["chunks", "fused", "fold"], default="chunks",
                     help="how a chunked workload's step runs: pa_attn_fwd per chunk + pa_attn_merge, one "
-                         "pa_attn_fwd_chunks launch, or pa_attn_fwd_accum folds")
+                         "pa_attn_fwd_chunks launch, or pa_attn_fwd_accum folds; with the ring or USP over "
+                         "several GPUs, chunks = per-block partials + one merge, fold = the fp32 running state")
     ap.add_argument("--fp8", action="store_true",
                     help="time the e4m3 forward (pa_attn_fwd_fp8) instead of bf16; one-chunk workloads")
     ap.add_argument("--heads", type=int, default=None,

@@ -63,8 +63,19 @@ def _default_attend(q, k, v, o_acc, lse_acc, first, final, out, scale):
     attn_fwd_accum(q, k, v, o_acc, lse_acc, first=first, final=final, out=out, scale=scale)
 
 
+def _default_attend_part(q, k, v, o_part, lse_part, scale):
+    from ._binding import attn_fwd
+    attn_fwd(q, k, v, scale=scale, out=o_part, lse=lse_part)
+
+
+def _default_merge(o_parts, lse_parts, out, lse):
+    from ._binding import attn_merge
+    attn_merge(o_parts, lse_parts, out=out, lse=lse)
+
+
 def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None, scale: Optional[float] = None,
-                   out=None, attend: Optional[Callable] = None, comm_stream=None, trace: Optional[list] = None):
+                   out=None, attend: Optional[Callable] = None, comm_stream=None, trace: Optional[list] = None,
+                   partials: bool = False, attend_part: Optional[Callable] = None, merge: Optional[Callable] = None):
     """Ring attention of this rank's queries over every rank's K/V block.
 
     q [B,H,n_q,d] and k, v [B,H,n_kv,d] are this rank's blocks (bf16 CUDA
@@ -72,7 +83,16 @@ def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
     block length (gathered from the ranks when not given).  Returns
     (o [B,H,n_q,d], lse [B,H,n_q] fp32): this rank's queries attended over
     the whole sequence.  ``trace``, if a list, receives one entry per step
-    (the schedule as executed)."""
+    (the schedule as executed).
+
+    Each step folds the block it holds into an fp32 running (O, LSE)
+    (``attend``: the accumulate launch).  With ``partials`` each step instead
+    writes the block's own partial (O in q's dtype, LSE) with the plain
+    forward (``attend_part``), and one LSE merge (``merge``) combines the
+    world-size partials after the last step: the per-step launches skip the
+    state's read and write, at the price of one partial per rank held until
+    the end and O rounded once per block (the same result up to that
+    rounding; the merge is exact in the pages' sense)."""
     import math
 
     import torch
@@ -99,12 +119,29 @@ def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
     # The running state is fp32 for the library's kernels; CPU tensors (the
     # exchange tests) keep at least their own precision.
     state_dtype = torch.float32 if cuda else torch.promote_types(q.dtype, torch.float32)
-    o_acc = torch.empty((B, H, n_q, d), dtype=state_dtype, device=q.device)
     lse_acc = torch.empty((B, H, n_q), dtype=state_dtype, device=q.device)
     if out is None:
         out = torch.empty_like(q)
+    if partials:
+        attend_part = attend_part or _default_attend_part
+        merge = merge or _default_merge
+        o_parts = torch.empty((world, B, H, n_q, d), dtype=q.dtype, device=q.device)
+        lse_parts = torch.empty((world, B, H, n_q), dtype=state_dtype, device=q.device)
+        o_acc = None
+    else:
+        o_acc = torch.empty((B, H, n_q, d), dtype=state_dtype, device=q.device)
+
+    def step_attend(s, kk, vv):
+        if partials:
+            if world == 1:
+                attend_part(q, kk, vv, out, lse_acc, scale)
+            else:
+                attend_part(q, kk, vv, o_parts[s], lse_parts[s], scale)
+        else:
+            attend(q, kk, vv, o_acc, lse_acc, s == 0, s == world - 1, out if s == world - 1 else None, scale)
+
     if world == 1:
-        attend(q, k, v, o_acc, lse_acc, True, True, out, scale)
+        step_attend(0, k, v)
         if trace is not None:
             trace.append({"step": 0, "block": 0})
         return out, lse_acc
@@ -151,7 +188,7 @@ def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
                     recv_done.record(comm)
             else:
                 reqs = dist.batch_isend_irecv(ops)
-        attend(q, cur_k, cur_v, o_acc, lse_acc, s == 0, s == world - 1, out if s == world - 1 else None, scale)
+        step_attend(s, cur_k, cur_v)
         if trace is not None:
             trace.append({"step": s, "block": ent["block"], "n_keys": int(cur_k.shape[2])})
         if s < world - 1:
@@ -163,6 +200,8 @@ def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
                 for r in reqs:
                     r.wait()
             cur_k, cur_v = nxt
+    if partials:
+        merge(o_parts, lse_parts, out, lse_acc)
     if cuda:
         # Work after this call (and the receive buffers' release) comes after
         # everything the comm stream did.
@@ -262,12 +301,14 @@ def usp_groups(ulysses_degree: int, group=None):
 
 
 def usp_attention(q, k, v, ulysses_group, ring_group, scale: Optional[float] = None, attend: Optional[Callable] = None,
-                  comm_stream=None, trace: Optional[list] = None):
+                  comm_stream=None, trace: Optional[list] = None, partials: bool = False,
+                  attend_part: Optional[Callable] = None, merge: Optional[Callable] = None):
     """Unified (Ulysses x ring) attention of this rank's sequence shard q, k, v
     [B,H,n,d] (the same n and H on every rank; H divisible by the Ulysses
     degree) over the whole sequence, which is sharded over the ranks in
     group-rank order (see usp_groups).  Returns (o [B,H,n,d], lse [B,H,n]).
-    ``attend`` is the fold step passed to ring_attention."""
+    ``attend``, ``partials``, ``attend_part`` and ``merge`` are passed to
+    ring_attention."""
     import math
 
     import torch.distributed as dist
@@ -284,5 +325,6 @@ def usp_attention(q, k, v, ulysses_group, ring_group, scale: Optional[float] = N
     qh, kh, vh = (_seq_to_heads(t, ulysses_group) for t in (q, k, v))   # [B, H/U, U*n, d]
     out = qh.new_empty(qh.shape)
     o_h, lse_h = ring_attention(qh, kh, vh, group=ring_group, kv_lens=[U * n] * R, scale=scale, out=out,
-                                attend=attend, comm_stream=comm_stream, trace=trace)
+                                attend=attend, comm_stream=comm_stream, trace=trace, partials=partials,
+                                attend_part=attend_part, merge=merge)
     return _heads_to_seq(o_h, ulysses_group), _heads_to_seq(lse_h, ulysses_group)

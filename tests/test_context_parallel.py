@@ -76,6 +76,58 @@ def _ring_rank(rank, world, port, q_lens, kv_lens, gather, out_q):
         dist.destroy_process_group()
 
 
+def _oracle_part(q, k, v, o_part, lse_part, scale):
+    """One block's partial (O, LSE), from the oracle."""
+    o_b, l_b = oracle.attention(q, k, v, scale)
+    o_part.copy_(torch.from_numpy(o_b))
+    lse_part.copy_(torch.from_numpy(l_b))
+
+
+def _ring_partials_rank(rank, world, port, q_lens, kv_lens, out_q):
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import ring_attention
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        q, k, v = _global_case(6, 2, 3, max(sum(q_lens), sum(kv_lens)), 8)
+        qs = np.cumsum([0] + list(q_lens))
+        ks = np.cumsum([0] + list(kv_lens))
+        q_r = q[:, :, qs[rank]:qs[rank + 1]].contiguous()
+        k_r = k[:, :, ks[rank]:ks[rank + 1]].contiguous()
+        v_r = v[:, :, ks[rank]:ks[rank + 1]].contiguous()
+        trace, merged = [], []
+
+        def merge(o_parts, lse_parts, out, lse):
+            merged.append(o_parts.shape[0])
+            o_m, l_m = oracle.merge(o_parts.numpy(), lse_parts.numpy())
+            out.copy_(torch.from_numpy(o_m))
+            lse.copy_(torch.from_numpy(l_m))
+
+        out, lse = ring_attention(q_r, k_r, v_r, scale=SCALE, out=torch.empty_like(q_r), partials=True,
+                                  attend_part=_oracle_part, merge=merge, trace=trace)
+        o_ref, l_ref = oracle.attention(q_r, k[:, :, :ks[-1]], v[:, :, :ks[-1]], SCALE)
+        out_q.put((rank, float(np.abs(out.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()),
+                   trace, merged))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("q_lens,kv_lens", [((6, 6), (6, 6)), ((5, 9, 4), (7, 3, 11))])
+def test_ring_attention_partials_gloo(q_lens, kv_lens):
+    """The partials form of the ring (diffusers "Context parallelism", section
+    "Ring Attention": once the ring has gone round, the blocks' partials
+    combine into the exact result): every block's partial once, one merge of
+    world-size parts, the whole-sequence attention on every rank."""
+    world = len(q_lens)
+    got = _run(_ring_partials_rank, world, q_lens, kv_lens)
+    for rank in range(world):
+        err_o, err_l, trace, merged = got[rank]
+        assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
+        assert [t["block"] for t in trace] == [(rank - s) % world for s in range(world)]
+        assert [t["n_keys"] for t in trace] == [kv_lens[(rank - s) % world] for s in range(world)]
+        assert merged == [world]
+
+
 def _subgroup_rank(rank, world, port, out_q):
     """Ranks 0 and 2 of a 3-rank world run the ring in a subgroup; rank 1 only
     joins the group creation (a collective over the world)."""
@@ -197,7 +249,7 @@ def test_ulysses_attention_gloo(world, H):
         assert seen == [(2, H // world, n * world, 8)]     # its heads, the whole sequence
 
 
-def _usp_rank(rank, world, port, U, n, H, out_q):
+def _usp_rank(rank, world, port, U, n, H, partials, out_q):
     import torch.distributed as dist
     from context_blocks_b200.context_parallel import usp_attention, usp_groups
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
@@ -206,8 +258,17 @@ def _usp_rank(rank, world, port, U, n, H, out_q):
         q, k, v = _global_case(9, 2, H, n * world, 8)
         sl = slice(rank * n, (rank + 1) * n)
         trace = []
-        o, lse = usp_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
-                               ug, rg, scale=SCALE, attend=_oracle_fold, trace=trace)
+        if partials:
+            def merge(o_parts, lse_parts, out, lse):
+                o_m, l_m = oracle.merge(o_parts.numpy(), lse_parts.numpy())
+                out.copy_(torch.from_numpy(o_m))
+                lse.copy_(torch.from_numpy(l_m))
+            o, lse = usp_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
+                                   ug, rg, scale=SCALE, trace=trace, partials=True, attend_part=_oracle_part,
+                                   merge=merge)
+        else:
+            o, lse = usp_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
+                                   ug, rg, scale=SCALE, attend=_oracle_fold, trace=trace)
         o_ref, l_ref = oracle.attention(q[:, :, sl], k, v, SCALE)
         out_q.put((rank, float(np.abs(o.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()),
                    [t["block"] for t in trace], dist.get_world_size(ug), dist.get_world_size(rg)))
@@ -216,13 +277,13 @@ def _usp_rank(rank, world, port, U, n, H, out_q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("U", [1, 2, 4])
-def test_usp_attention_gloo(U):
+@pytest.mark.parametrize("U,partials", [(1, False), (2, False), (4, False), (2, True)])
+def test_usp_attention_gloo(U, partials):
     """diffusers "Context parallelism", section "Unified Attention": 4 ranks
     as a Ulysses x ring grid (4 x 1, 2 x 2, 1 x 4); every rank gets the
     attention of its queries over the whole sequence."""
     world, n, H = 4, 3, 4
-    got = _run(_usp_rank, world, U, n, H)
+    got = _run(_usp_rank, world, U, n, H, partials)
     R = world // U
     for rank in range(world):
         err_o, err_l, blocks, u_size, r_size = got[rank]
@@ -230,3 +291,25 @@ def test_usp_attention_gloo(U):
         assert (u_size, r_size) == (U, R)
         g = rank // U
         assert blocks == [(g - s) % R for s in range(R)]     # the ring runs across the groups
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("partials", [False, True])
+def test_ring_attention_one_rank_library_kernels(partials):
+    """A one-rank group on the GPU: ring_attention with the library's own
+    step (the fp32 fold, or a block partial) against the oracle."""
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import ring_attention
+    from tests._parity import assert_close
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    try:
+        g = torch.Generator(device="cuda").manual_seed(31)
+        q, k, v = (torch.randn((1, 3, n, 128), generator=g, device="cuda").to(torch.bfloat16)
+                   for n in (300, 517, 517))
+        scale = 128 ** -0.5   # the bars of the GPU parity tests are set for 1/sqrt(d)
+        o, lse = ring_attention(q, k, v, kv_lens=[517], scale=scale, partials=partials)
+        torch.cuda.synchronize()
+        o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), scale)
+        assert_close(o, lse, o_ref, l_ref, f"ring one rank, partials={partials}")
+    finally:
+        dist.destroy_process_group()
