@@ -98,19 +98,41 @@ def _basis(peaks) -> str:
     """Where the peak figures came from, for the JSON line."""
     if peaks["source"] == "measured":
         return "measured burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
+    if peaks["source"] == "unreadable":
+        return "fallback burst bf16 of the profiling recipe (MEASURED_PEAKS.json present, without hbm_gbs / bf16_tflops)"
     return "fallback burst bf16 of the profiling recipe (MEASURED_PEAKS.json absent on this machine)"
+
+
+def _find_key(d, key):
+    """The first value stored under `key` in a JSON object, searching nested
+    objects breadth-first (the file's exact nesting is not fixed here)."""
+    todo = [d]
+    while todo:
+        x = todo.pop(0)
+        if isinstance(x, dict):
+            if key in x and isinstance(x[key], (int, float)):
+                return float(x[key])
+            todo.extend(x.values())
+        elif isinstance(x, list):
+            todo.extend(x)
+    return None
 
 
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(path):
+        return dict(FALLBACK_PEAKS, source="fallback")
     try:
         with open(path) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
-                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                "source": "measured"}
     except Exception:
-        return dict(FALLBACK_PEAKS, source="fallback")
+        return dict(FALLBACK_PEAKS, source="unreadable")
+    hbm, bf16 = _find_key(d, "hbm_gbs"), _find_key(d, "bf16_tflops")
+    if hbm is None or bf16 is None or hbm <= 0 or bf16 <= 0:
+        return dict(FALLBACK_PEAKS, source="unreadable")
+    sus = _find_key(d, "bf16_tflops_sustained")
+    return {"hbm_gbs": hbm, "bf16_tflops": bf16, "bf16_tflops_sustained": sus if sus and sus > 0 else bf16,
+            "source": "measured"}
 
 
 # --------------------------------------------------------------------- clocks

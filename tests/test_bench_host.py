@@ -151,3 +151,21 @@ def test_ring_shard_sizes_cover_the_sequence():
         assert len(sizes) == world and sum(sizes) == n
         assert max(sizes) - min(sizes) <= 1
         assert sizes == sorted(sizes, reverse=True)
+
+
+def test_peaks_file_nested_missing_and_absent(tmp_path, monkeypatch):
+    """The peak figures come from MEASURED_PEAKS.json at any nesting; a file
+    without them, or no file, falls back to the recipe's figures and says so."""
+    import json
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p = bench._peaks()
+    assert p["source"] == "fallback" and p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    assert "absent" in bench._basis(p)
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"box": {"hbm_gbs": 6547.5, "gemm": {"bf16_tflops": 1674.6, "bf16_tflops_sustained": 1363.4}}}))
+    p = bench._peaks()
+    assert p == {"hbm_gbs": 6547.5, "bf16_tflops": 1674.6, "bf16_tflops_sustained": 1363.4, "source": "measured"}
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6547.5}))
+    p = bench._peaks()
+    assert p["source"] == "unreadable" and "present" in bench._basis(p)
