@@ -716,8 +716,11 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
 
     ws, rank = dist.get_world_size(), dist.get_rank()
     nq_all, nk_all = shard_sizes(w.Nq, ws), shard_sizes(w.Nk, ws)
-    if ulysses and (len(set(nq_all)) > 1 or nq_all != nk_all or w.H % ws):
-        raise SystemExit(f"--parallel ulysses needs Nq = Nk divisible by {ws} and heads divisible by {ws}")
+    if ulysses and nq_all != nk_all:
+        raise SystemExit("--parallel ulysses needs Nq = Nk: each rank holds the same tokens of q, k and v")
+    # Shards of different lengths or heads that do not divide over the ranks:
+    # Ulysses Anything (per-peer pieces of different sizes in the all-to-alls).
+    anything = ulysses and (len(set(nq_all)) > 1 or w.H % ws != 0)
     if usp_degree and (len(set(nq_all)) > 1 or nq_all != nk_all or w.H % usp_degree or ws % usp_degree):
         raise SystemExit(f"--parallel usp needs Nq = Nk divisible by {ws}, and heads and {ws} ranks divisible by "
                          f"the Ulysses degree {usp_degree}")
@@ -749,6 +752,9 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
         return res
 
     def step(timed=False):
+        if anything:
+            return cp.ulysses_anything_attention(q, k, v, seq_lens=nq_all, scale=w.scale,
+                                                 attend_full=attend_full_timed if timed else None)
         if ulysses:
             return cp.ulysses_attention(q, k, v, scale=w.scale, attend_full=attend_full_timed if timed else None)
         if usp_degree:
@@ -780,13 +786,17 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
     value = fl * args.steps / (max_ms * 1e-3) / 1e12
     fwd_ms = [a.elapsed_time(b) for a, b in zip(*fwd_ev)]
     # the forward kernel (the fold, or the plain forward of a block's partial):
-    # this rank's FLOPs per ring pass over its launches
-    fl_rank = workloads.flops(w.B, w.H, nq_all[rank], w.Nk, w.d)
-    launch_ms = statistics.fmean(fwd_ms)
+    # this rank's FLOPs per ring pass over its launches; with Ulysses, its
+    # heads over the whole sequence
+    fl_rank = (workloads.flops(w.B, cp.head_split(w.H, ws)[0][rank], w.Nq, w.Nk, w.d) if ulysses
+               else workloads.flops(w.B, w.H, nq_all[rank], w.Nk, w.d))
+    # (a Ulysses Anything rank that holds no head launches nothing)
+    launch_ms = statistics.fmean(fwd_ms) if fwd_ms else 0.0
     # ring: one fold launch per block, 1/ws of the rank's FLOPs each; Ulysses:
     # one launch over the rank's heads and the whole sequence; USP: one fold
     # per ring step, 1/ring_len of the rank's FLOPs each
-    achieved = (fl_rank / ring_len if not ulysses else fl_rank) / (launch_ms * 1e-3) / 1e12
+    achieved = ((fl_rank / ring_len if not ulysses else fl_rank) / (launch_ms * 1e-3) / 1e12
+                if launch_ms > 0 else 0.0)
     peak = peaks["bf16_tflops"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": None,
@@ -821,7 +831,10 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(_config(w, parallelism=(f"Ulysses attention over {ws} ranks (two NCCL all-to-alls)" if ulysses
+            "config": dict(_config(w, parallelism=(f"Ulysses Anything attention over {ws} ranks (two NCCL all-to-alls "
+                                                   f"with per-peer pieces; uneven shards or heads)" if anything
+                                                   else f"Ulysses attention over {ws} ranks (two NCCL all-to-alls)"
+                                                   if ulysses
                                                    else f"USP over {ws} ranks: Ulysses degree {usp_degree} x ring "
                                                         f"degree {ring_len}" + _ring_how(partials) if usp_degree
                                                    else f"ring attention over {ws} ranks (NCCL P2P on a second "

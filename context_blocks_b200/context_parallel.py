@@ -36,7 +36,8 @@ from __future__ import annotations
 
 from typing import Callable, List, Optional, Sequence
 
-__all__ = ["ring_schedule", "ring_attention", "ulysses_attention", "usp_groups", "usp_attention"]
+__all__ = ["ring_schedule", "ring_attention", "ulysses_attention", "ulysses_anything_attention", "head_split",
+           "usp_groups", "usp_attention"]
 
 
 def ring_schedule(rank: int, world: int) -> List[dict]:
@@ -268,6 +269,105 @@ def ulysses_attention(q, k, v, group=None, scale: Optional[float] = None, attend
     qh, kh, vh = _seq_to_heads(q, group), _seq_to_heads(k, group), _seq_to_heads(v, group)
     o_h, lse_h = attend_full(qh, kh, vh, scale)
     return _heads_to_seq(o_h, group), _heads_to_seq(lse_h, group)
+
+
+def head_split(H: int, P: int):
+    """Heads per rank for Ulysses Anything: contiguous groups in rank order,
+    the first H mod P ranks taking one more head (some ranks get none when
+    H < P).  Returns (sizes, starts)."""
+    base, extra = divmod(H, P)
+    sizes = [base + (1 if r < extra else 0) for r in range(P)]
+    starts = [sum(sizes[:r]) for r in range(P)]
+    return sizes, starts
+
+
+def _a2a_var(send_parts, recv_numels, group, like):
+    """all_to_all with a flat piece per peer: send_parts[s] goes to rank s,
+    and the piece from rank s has recv_numels[s] elements."""
+    import torch
+    import torch.distributed as dist
+    send = torch.cat([x.reshape(-1) for x in send_parts]) if send_parts else like.new_empty(0)
+    recv = like.new_empty(sum(recv_numels))
+    dist.all_to_all_single(recv, send, output_split_sizes=list(recv_numels),
+                           input_split_sizes=[x.numel() for x in send_parts], group=group)
+    return torch.split(recv, list(recv_numels))
+
+
+def _seq_to_heads_any(x, group, seq_lens, sizes, starts):
+    """[B, H, n_r, ...] sequence shard -> [B, h_r, sum(seq_lens), ...]: rank
+    s's head group goes to rank s; the shards line up along the sequence in
+    rank order."""
+    import torch
+    import torch.distributed as dist
+    r = dist.get_rank(group)
+    B = x.shape[0]
+    rest = tuple(x.shape[3:])
+    e = 1
+    for t in rest:
+        e *= t
+    send = [x[:, h0:h0 + hs] for h0, hs in zip(starts, sizes)]
+    pieces = _a2a_var(send, [B * sizes[r] * n_s * e for n_s in seq_lens], group, x)
+    parts = [pc.view(B, sizes[r], n_s, *rest) for pc, n_s in zip(pieces, seq_lens)]
+    return torch.cat(parts, dim=2).contiguous()
+
+
+def _heads_to_seq_any(y, group, seq_lens, sizes):
+    """The inverse of _seq_to_heads_any: [B, h_r, sum(seq_lens), ...] ->
+    [B, H, n_r, ...]."""
+    import torch
+    import torch.distributed as dist
+    r = dist.get_rank(group)
+    B = y.shape[0]
+    rest = tuple(y.shape[3:])
+    e = 1
+    for t in rest:
+        e *= t
+    offs = [sum(seq_lens[:s]) for s in range(len(seq_lens))]
+    send = [y[:, :, o:o + n_s] for o, n_s in zip(offs, seq_lens)]
+    pieces = _a2a_var(send, [B * h_s * seq_lens[r] * e for h_s in sizes], group, y)
+    parts = [pc.view(B, h_s, seq_lens[r], *rest) for pc, h_s in zip(pieces, sizes)]
+    return torch.cat(parts, dim=1).contiguous()
+
+
+def ulysses_anything_attention(q, k, v, group=None, seq_lens: Optional[Sequence[int]] = None,
+                               scale: Optional[float] = None, attend_full: Optional[Callable] = None):
+    """Ulysses attention without divisibility (diffusers "Context
+    parallelism", section "Ulysses Anything"): this rank's sequence shard q,
+    k, v [B,H,n_r,d] in, where the shard lengths may differ between ranks
+    (``seq_lens``, gathered when not given) and H need not divide by the rank
+    count (head_split); this rank's shard of the output (o [B,H,n_r,d],
+    lse [B,H,n_r]) out.  The two all-to-alls carry per-peer pieces of
+    different sizes; a rank that holds no head computes nothing."""
+    import math
+
+    import torch
+    import torch.distributed as dist
+
+    P = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    B, H, n, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("Ulysses needs q, k, v of one shape [B,H,n,d] on each rank")
+    if seq_lens is None:
+        t = torch.tensor([n], dtype=torch.int64, device=q.device)
+        lens = [torch.zeros_like(t) for _ in range(P)]
+        dist.all_gather(lens, t, group=group)
+        seq_lens = [int(x.item()) for x in lens]
+    seq_lens = [int(x) for x in seq_lens]
+    if len(seq_lens) != P or seq_lens[r] != n or min(seq_lens) < 1:
+        raise ValueError(f"seq_lens {seq_lens} does not match the group ({P} ranks, own shard {n})")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    attend_full = attend_full or _default_attend_full
+    sizes, starts = head_split(H, P)
+    qh, kh, vh = (_seq_to_heads_any(x, group, seq_lens, sizes, starts) for x in (q, k, v))
+    if sizes[r] > 0:
+        o_h, lse_h = attend_full(qh, kh, vh, scale)
+    else:
+        lse_dtype = torch.float32 if q.is_cuda else torch.promote_types(q.dtype, torch.float32)
+        o_h = qh.new_empty((B, 0, sum(seq_lens), d))
+        lse_h = torch.empty((B, 0, sum(seq_lens)), dtype=lse_dtype, device=q.device)
+    return _heads_to_seq_any(o_h, group, seq_lens, sizes), _heads_to_seq_any(lse_h, group, seq_lens, sizes)
 
 
 def usp_groups(ulysses_degree: int, group=None):

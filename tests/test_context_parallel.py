@@ -249,6 +249,48 @@ def test_ulysses_attention_gloo(world, H):
         assert seen == [(2, H // world, n * world, 8)]     # its heads, the whole sequence
 
 
+def _ulysses_anything_rank(rank, world, port, lens, H, gather, out_q):
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import head_split, ulysses_anything_attention
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        q, k, v = _global_case(8, 2, H, sum(lens), 8)
+        off = np.cumsum([0] + list(lens))
+        sl = slice(int(off[rank]), int(off[rank + 1]))
+        seen = []
+
+        def attend_full(qh, kh, vh, scale):
+            seen.append(tuple(qh.shape))
+            o, l = oracle.attention(qh, kh, vh, scale)
+            return torch.from_numpy(o), torch.from_numpy(l)
+
+        o, lse = ulysses_anything_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                                            v[:, :, sl].contiguous(), seq_lens=None if gather else lens,
+                                            scale=SCALE, attend_full=attend_full)
+        o_ref, l_ref = oracle.attention(q[:, :, sl], k, v, SCALE)
+        out_q.put((rank, float(np.abs(o.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()),
+                   tuple(o.shape), seen, head_split(H, world)[0][rank]))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("lens,H,gather", [((5, 9), 3, False), ((5, 9, 4), 5, True), ((4, 1, 7), 2, False),
+                                           ((6, 6), 4, True)])
+def test_ulysses_anything_attention_gloo(lens, H, gather):
+    """diffusers "Context parallelism", section "Ulysses Anything": shards of
+    different lengths and a head count that need not divide by the ranks
+    (with 3 ranks and 2 heads one rank holds none); every rank gets its own
+    queries attended over the whole sequence."""
+    world = len(lens)
+    got = _run(_ulysses_anything_rank, world, lens, H, gather)
+    for rank in range(world):
+        err_o, err_l, shape, seen, heads = got[rank]
+        assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
+        assert shape == (2, H, lens[rank], 8)
+        assert seen == ([(2, heads, sum(lens), 8)] if heads else [])
+
+
 def _usp_rank(rank, world, port, U, n, H, partials, out_q):
     import torch.distributed as dist
     from context_blocks_b200.context_parallel import usp_attention, usp_groups
@@ -313,3 +355,13 @@ def test_ring_attention_one_rank_library_kernels(partials):
         assert_close(o, lse, o_ref, l_ref, f"ring one rank, partials={partials}")
     finally:
         dist.destroy_process_group()
+
+
+def test_head_split_covers_every_head_once():
+    from context_blocks_b200.context_parallel import head_split
+    for H in range(1, 30):
+        for P in range(1, 9):
+            sizes, starts = head_split(H, P)
+            assert sum(sizes) == H and len(sizes) == P
+            assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+            assert starts == [sum(sizes[:r]) for r in range(P)]
