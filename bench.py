@@ -618,9 +618,10 @@ def run_ours(args):
     peaks = _peaks()
     sampler = ClockSampler(local)
     fp8 = bool(getattr(args, "fp8", False))
-    if ws > 1 and args.parallel in ("ring", "ulysses", "usp"):
+    if ws > 1 and args.parallel in ("ring", "ulysses", "usp", "ring_anything"):
         return run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=(args.parallel == "ulysses"),
-                        usp_degree=(args.ulysses_degree if args.parallel == "usp" else 0))
+                        usp_degree=(args.ulysses_degree if args.parallel == "usp" else 0),
+                        gather=(args.parallel == "ring_anything"))
     mode = args.mode if len(w.chunks) > 1 else "chunks"
     res = time_workload(pa, w, args.steps, args.warmup, device, sampler=sampler, barrier=barrier, fp8=fp8, mode=mode)
     if res["status"] != 0:
@@ -700,7 +701,7 @@ def _ring_how(partials: bool) -> str:
             else "; per-block folds into an fp32 state (pa_attn_fwd_accum)")
 
 
-def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_degree=0):
+def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_degree=0, gather=False):
     """Context parallelism over the process group: rank r holds shard r of
     the query rows and of the K/V rows of workload `w` and runs
     context_parallel.ring_attention (or, with ``ulysses``, the all-to-all
@@ -724,9 +725,9 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
     if usp_degree and (len(set(nq_all)) > 1 or nq_all != nk_all or w.H % usp_degree or ws % usp_degree):
         raise SystemExit(f"--parallel usp needs Nq = Nk divisible by {ws}, and heads and {ws} ranks divisible by "
                          f"the Ulysses degree {usp_degree}")
-    if args.mode == "fused" and not ulysses:
+    if args.mode == "fused" and not ulysses and not gather:
         raise SystemExit("--mode fused is a one-GPU mode: the ring's blocks arrive one at a time")
-    partials = not ulysses and args.mode == "chunks"
+    partials = not ulysses and not gather and args.mode == "chunks"
     groups = cp.usp_groups(usp_degree) if usp_degree else None
     ring_len = ws // usp_degree if usp_degree else ws
     wr = dataclasses.replace(w, Nq=nq_all[rank], Nk=nk_all[rank], chunks=(nk_all[rank],), seed=w.seed + 100 * rank)
@@ -745,6 +746,12 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
         pa.attn_fwd(qq, kk, vv, scale=scale, out=o_part, lse=lse_part)
         fwd_ev[1].append(_record())
 
+    def attend_chunks_timed(qq, kcs, vcs, scale):
+        fwd_ev[0].append(_record())
+        res = cp._default_attend_chunks(qq, kcs, vcs, scale)
+        fwd_ev[1].append(_record())
+        return res
+
     def attend_full_timed(qq, kk, vv, scale):
         fwd_ev[0].append(_record())
         res = pa.attn_fwd(qq, kk, vv, scale=scale)
@@ -752,6 +759,9 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
         return res
 
     def step(timed=False):
+        if gather:
+            return cp.ring_anything_attention(q, k, v, kv_lens=nk_all, scale=w.scale,
+                                              attend_chunks=attend_chunks_timed if timed else None)
         if anything:
             return cp.ulysses_anything_attention(q, k, v, seq_lens=nq_all, scale=w.scale,
                                                  attend_full=attend_full_timed if timed else None)
@@ -795,12 +805,12 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
     # ring: one fold launch per block, 1/ws of the rank's FLOPs each; Ulysses:
     # one launch over the rank's heads and the whole sequence; USP: one fold
     # per ring step, 1/ring_len of the rank's FLOPs each
-    achieved = ((fl_rank / ring_len if not ulysses else fl_rank) / (launch_ms * 1e-3) / 1e12
+    achieved = ((fl_rank if ulysses or gather else fl_rank / ring_len) / (launch_ms * 1e-3) / 1e12
                 if launch_ms > 0 else 0.0)
     peak = peaks["bf16_tflops"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": None,
-            "kernel": f"attn_fwd_kernel<{w.d}, false, {'false' if ulysses or partials else 'true'}>",
+            "kernel": f"attn_fwd_kernel<{w.d}, false, {'false' if ulysses or partials or gather else 'true'}>",
             "launch_ms": launch_ms,
             "peak_basis": f"{_basis(peaks)}, rank {rank}"}
     # End to end: each step uploads this rank's shards from pinned host
@@ -835,6 +845,8 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
                                                    f"with per-peer pieces; uneven shards or heads)" if anything
                                                    else f"Ulysses attention over {ws} ranks (two NCCL all-to-alls)"
                                                    if ulysses
+                                                   else f"Ring Anything over {ws} ranks (padded K/V blocks all-gathered, "
+                                                        f"trimmed, one fused pa_attn_fwd_chunks launch)" if gather
                                                    else f"USP over {ws} ranks: Ulysses degree {usp_degree} x ring "
                                                         f"degree {ring_len}" + _ring_how(partials) if usp_degree
                                                    else f"ring attention over {ws} ranks (NCCL P2P on a second "
@@ -842,7 +854,8 @@ def run_ring(args, pa, w, peaks, sampler, device, barrier, ulysses=False, usp_de
                            q_shards=nq_all, kv_shards=nk_all,
                            l2="each rank's K/V blocks rotate through the ring; inputs far larger than L2"),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak, "roofline": roof, "clocks": sampler.summary(),
-            "gpu_launches": args.steps * (1 if ulysses else ring_len + (1 if partials else 0)),
+            "gpu_launches": args.steps * (1 if ulysses or (gather and ws <= 8)
+                                          else ws + 1 if gather else ring_len + (1 if partials else 0)),
             "e2e": {"value": fl * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
                     "d2h_bytes_per_step": int(out.numel() * 2 + out.numel() // w.d * 4), "steps": e_steps,
@@ -1061,9 +1074,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="hunyuan", choices=sorted(workloads.WORKLOADS))
-    ap.add_argument("--parallel", choices=["ring", "ulysses", "usp", "replicas"], default="ring",
+    ap.add_argument("--parallel", choices=["ring", "ulysses", "usp", "ring_anything", "replicas"], default="ring",
                     help="with more than one GPU: ring, Ulysses or USP (Ulysses x ring) attention over the ranks, "
-                         "or independent replicas")
+                         "Ring Anything (padded all-gather + one fused launch), or independent replicas")
     ap.add_argument("--ulysses-degree", type=int, default=2,
                     help="with --parallel usp: ranks per Ulysses group (the ring runs across the groups)")
     ap.add_argument("--mode", choices=["chunks", "fused", "fold"], default="chunks",

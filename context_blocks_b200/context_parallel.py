@@ -36,8 +36,8 @@ from __future__ import annotations
 
 from typing import Callable, List, Optional, Sequence
 
-__all__ = ["ring_schedule", "ring_attention", "ulysses_attention", "ulysses_anything_attention", "head_split",
-           "usp_groups", "usp_attention"]
+__all__ = ["ring_schedule", "ring_attention", "ring_anything_attention", "ulysses_attention",
+           "ulysses_anything_attention", "head_split", "usp_groups", "usp_attention"]
 
 
 def ring_schedule(rank: int, world: int) -> List[dict]:
@@ -208,6 +208,59 @@ def ring_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
         # everything the comm stream did.
         compute.wait_stream(comm)
     return out, lse_acc
+
+
+def _default_attend_chunks(q, k_chunks, v_chunks, scale):
+    from ._binding import attn_fwd_chunks
+    from .ring import blockwise_attention
+    if len(k_chunks) <= 8:
+        return attn_fwd_chunks(q, k_chunks, v_chunks, scale=scale)
+    return blockwise_attention(q, k_chunks, v_chunks, scale=scale)
+
+
+def ring_anything_attention(q, k, v, group=None, kv_lens: Optional[Sequence[int]] = None,
+                            scale: Optional[float] = None, attend_chunks: Optional[Callable] = None):
+    """Ring Anything (diffusers "Context parallelism", section "Ring Anything
+    Attention"): every rank pads its K/V block to the longest block, the
+    padded blocks are all-gathered, and each is trimmed back to its real
+    length before attention, so padding never enters the softmax.  Here the
+    trimmed blocks are the chunks of one launch (``attend_chunks``; by
+    default pa_attn_fwd_chunks for up to 8 ranks, per-block forwards + merge
+    beyond).  Returns (o [B,H,n_q,d], lse [B,H,n_q]) like ring_attention."""
+    import math
+
+    import torch
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, H, n_q, d = q.shape
+    if k.shape != v.shape or tuple(k.shape[:2]) != (B, H) or k.shape[3] != d:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    if kv_lens is None:
+        t = torch.tensor([k.shape[2]], dtype=torch.int64, device=q.device)
+        lens = [torch.zeros_like(t) for _ in range(world)]
+        dist.all_gather(lens, t, group=group)
+        kv_lens = [int(x.item()) for x in lens]
+    kv_lens = [int(x) for x in kv_lens]
+    if len(kv_lens) != world or kv_lens[rank] != k.shape[2] or min(kv_lens) < 1:
+        raise ValueError(f"kv_lens {kv_lens} does not match the group ({world} ranks, own block {k.shape[2]})")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    attend_chunks = attend_chunks or _default_attend_chunks
+    if world == 1:
+        return attend_chunks(q, [k], [v], scale)
+    m = max(kv_lens)
+    kv = torch.zeros((2, B, H, m, d), dtype=k.dtype, device=k.device)
+    kv[0, :, :, :k.shape[2]] = k
+    kv[1, :, :, :k.shape[2]] = v
+    gathered = [torch.empty_like(kv) for _ in range(world)]
+    dist.all_gather(gathered, kv, group=group)
+    # trimmed to each block's real length, as contiguous chunks
+    ks = [g[0, :, :, :n].contiguous() for g, n in zip(gathered, kv_lens)]
+    vs = [g[1, :, :, :n].contiguous() for g, n in zip(gathered, kv_lens)]
+    del gathered
+    return attend_chunks(q, ks, vs, scale)
 
 
 def _a2a(x, group):

@@ -291,6 +291,47 @@ def test_ulysses_anything_attention_gloo(lens, H, gather):
         assert seen == ([(2, heads, sum(lens), 8)] if heads else [])
 
 
+def _ring_anything_rank(rank, world, port, q_lens, kv_lens, out_q):
+    import torch.distributed as dist
+    from context_blocks_b200.context_parallel import ring_anything_attention
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        q, k, v = _global_case(10, 2, 3, max(sum(q_lens), sum(kv_lens)), 8)
+        qs = np.cumsum([0] + list(q_lens))
+        ks = np.cumsum([0] + list(kv_lens))
+        q_r = q[:, :, qs[rank]:qs[rank + 1]].contiguous()
+        k_r = k[:, :, ks[rank]:ks[rank + 1]].contiguous()
+        v_r = v[:, :, ks[rank]:ks[rank + 1]].contiguous()
+        seen = []
+
+        def attend_chunks(qq, k_chunks, v_chunks, scale):
+            seen.append([int(c.shape[2]) for c in k_chunks])
+            assert all(c.is_contiguous() for c in k_chunks + v_chunks)
+            o, l = oracle.attention(qq, torch.cat(k_chunks, dim=2), torch.cat(v_chunks, dim=2), scale)
+            return torch.from_numpy(o), torch.from_numpy(l)
+
+        o, lse = ring_anything_attention(q_r, k_r, v_r, scale=SCALE, attend_chunks=attend_chunks)
+        o_ref, l_ref = oracle.attention(q_r, k[:, :, :ks[-1]], v[:, :, :ks[-1]], SCALE)
+        out_q.put((rank, float(np.abs(o.numpy() - o_ref).max()), float(np.abs(lse.numpy() - l_ref).max()), seen))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("q_lens,kv_lens", [((6, 6), (6, 6)), ((5, 9, 4), (7, 3, 11))])
+def test_ring_anything_attention_gloo(q_lens, kv_lens):
+    """diffusers "Context parallelism", section "Ring Anything Attention":
+    blocks padded to the longest, all-gathered, trimmed back to their real
+    lengths (padding never enters the softmax), attended as one set of
+    chunks in rank order."""
+    world = len(q_lens)
+    got = _run(_ring_anything_rank, world, q_lens, kv_lens)
+    for rank in range(world):
+        err_o, err_l, seen = got[rank]
+        assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
+        assert seen == [list(kv_lens)]
+
+
 def _usp_rank(rank, world, port, U, n, H, partials, out_q):
     import torch.distributed as dist
     from context_blocks_b200.context_parallel import usp_attention, usp_groups
@@ -336,12 +377,13 @@ def test_usp_attention_gloo(U, partials):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("partials", [False, True])
+@pytest.mark.parametrize("partials", [False, True, "anything"])
 def test_ring_attention_one_rank_library_kernels(partials):
     """A one-rank group on the GPU: ring_attention with the library's own
-    step (the fp32 fold, or a block partial) against the oracle."""
+    step (the fp32 fold, or a block partial), and ring_anything_attention
+    with the fused chunk launch, against the oracle."""
     import torch.distributed as dist
-    from context_blocks_b200.context_parallel import ring_attention
+    from context_blocks_b200.context_parallel import ring_anything_attention, ring_attention
     from tests._parity import assert_close
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
     try:
@@ -349,7 +391,10 @@ def test_ring_attention_one_rank_library_kernels(partials):
         q, k, v = (torch.randn((1, 3, n, 128), generator=g, device="cuda").to(torch.bfloat16)
                    for n in (300, 517, 517))
         scale = 128 ** -0.5   # the bars of the GPU parity tests are set for 1/sqrt(d)
-        o, lse = ring_attention(q, k, v, kv_lens=[517], scale=scale, partials=partials)
+        if partials == "anything":
+            o, lse = ring_anything_attention(q, k, v, kv_lens=[517], scale=scale)
+        else:
+            o, lse = ring_attention(q, k, v, kv_lens=[517], scale=scale, partials=partials)
         torch.cuda.synchronize()
         o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), scale)
         assert_close(o, lse, o_ref, l_ref, f"ring one rank, partials={partials}")
