@@ -1055,6 +1055,25 @@ def extra_measurements(pa, device, peaks):
                             "gbs": 3.0 * x.numel() / (ms * 1e-3) / 1e9,
                             "frac_of_hbm": 3.0 * x.numel() / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     del x, q8
+    # First Block Cache's residual difference (pa_residual_diff) between two
+    # HunyuanVideo-sized first-block residuals (119056 tokens x 3072 channels
+    # bf16, 0.73 GB each, far above L2): algorithmic bytes = 4 per element
+    # (both read once); two inputs alternate so no call finds its data in L2.
+    n_res = 119056 * 3072
+    res = [torch.randn((n_res,), device=device).to(torch.bfloat16) for _ in range(3)]
+    rd_out = torch.empty((1,), dtype=torch.float32, device=device)
+    for i in range(3):
+        pa.residual_diff(res[i % 3], res[(i + 1) % 3], out=rd_out)
+    torch.cuda.synchronize()
+    t0.record()
+    for i in range(12):
+        pa.residual_diff(res[i % 3], res[(i + 1) % 3], out=rd_out)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / 12
+    out["residual_diff"] = {"elements": n_res, "ms": ms, "gbs": 4.0 * n_res / (ms * 1e-3) / 1e9,
+                            "frac_of_hbm": 4.0 * n_res / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del res
     w8 = workloads.get("hunyuan").with_chunks(workloads.HUNYUAN_CHUNKS8)
     r = time_workload(pa, w8, 2, 1, device)
     fl = workloads.flops(w8.B, w8.H, w8.Nq, w8.Nk, w8.d)

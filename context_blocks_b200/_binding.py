@@ -39,6 +39,7 @@ SIGNATURES = {
     "pa_attn_fwd_chunks": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
     "pa_attn_merge": (_I, [_VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _VP]),
     "pa_attn_chunks_noalloc": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
+    "pa_residual_diff": (_I, [_VP, _VP, ctypes.c_longlong, _VP, _VP]),
     "pa_status_string": (ctypes.c_char_p, [_I]),
     "pa_last_error": (ctypes.c_char_p, []),
     "pa_poll_device_status": (_I, []),
@@ -256,6 +257,28 @@ def quantize_e4m3(x, out=None, scale=None, stream=None, check: bool = False):
                                          _stream_handle(stream, x.device))
     _check(rc, "pa_quantize_e4m3", check)
     return out, scale
+
+
+def residual_diff(cur, prev, out=None, stream=None, check: bool = False):
+    """First Block Cache's residual difference (``pa_residual_diff``):
+    sum |cur - prev| / sum |prev| over two bf16 CUDA tensors of the same
+    shape, as a one-element float32 device tensor (no host synchronisation;
+    compare it with the threshold on the device or read it when needed)."""
+    import torch
+    for name, t in (("cur", cur), ("prev", prev)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.device.type != "cuda" \
+                or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous bfloat16 CUDA tensor")
+    if cur.shape != prev.shape:
+        raise ValueError(f"shape mismatch: cur {tuple(cur.shape)}, prev {tuple(prev.shape)}")
+    if out is None:
+        out = torch.empty((1,), dtype=torch.float32, device=cur.device)
+    elif out.dtype != torch.float32 or out.numel() != 1 or out.device != cur.device:
+        raise ValueError("out must be a one-element float32 tensor on cur's device")
+    rc = load_library().pa_residual_diff(cur.data_ptr(), prev.data_ptr(), cur.numel(), out.data_ptr(),
+                                         _stream_handle(stream, cur.device))
+    _check(rc, "pa_residual_diff", check)
+    return out
 
 
 def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None, check: bool = False):

@@ -16,6 +16,7 @@
 #include "quantize.cuh"
 #include "fwd_common.cuh"
 #include "lse_merge.cuh"
+#include "residual_diff.cuh"
 #include "pa_attn.h"
 
 namespace pa {
@@ -527,6 +528,37 @@ int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64) return launch_merge<64>(st, o_parts, lse_parts, n_parts, o, lse, rows, s);
   return launch_merge<128>(st, o_parts, lse_parts, n_parts, o, lse, rows, s);
+}
+
+int pa_residual_diff(const void* cur, const void* prev, long long n, float* out, void* stream) {
+  g_err[0] = '\0';
+  if (!cur || !prev || !out) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (n < 1) return fail(PA_ERR_INVALID_ARG, "n must be >= 1 (got %lld)", n);
+  if (!aligned(cur, 16) || !aligned(prev, 16)) return fail(PA_ERR_MISALIGNED, "cur and prev must be 16-byte aligned");
+  if (!aligned(out, 4)) return fail(PA_ERR_MISALIGNED, "out must be 4-byte aligned");
+  const uint64_t bytes = static_cast<uint64_t>(n) * 2;
+  if (overlap(cur, bytes, out, 4) || overlap(prev, bytes, out, 4))
+    return fail(PA_ERR_INVALID_ARG, "out overlaps an input");
+  (void)cudaGetLastError();
+  int dev = 0, rc;
+  const void* ptrs[3] = {cur, prev, out};
+  const char* names[3] = {"cur", "prev", "out"};
+  for (int i = 0; i < 3; ++i)
+    if ((rc = check_device_ptr(ptrs[i], names[i], &dev)) != PA_OK) return rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(dev, &st)) != PA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // A fixed grid for a given size and device (the result's rounding does not
+  // depend on scheduling): enough blocks to keep every SM streaming.
+  const long long vecs = (n / 8 + pa::kRdThreads - 1) / pa::kRdThreads;
+  const int grid = static_cast<int>(std::max<long long>(
+      1, std::min<long long>(vecs, std::min<long long>(4LL * st->sm_count, pa::kRdMaxBlocks))));
+  pa::residual_diff_partial_kernel<<<grid, pa::kRdThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(cur),
+                                                                   static_cast<const __nv_bfloat16*>(prev), n);
+  pa::residual_diff_final_kernel<<<1, pa::kRdThreads, 0, s>>>(grid, out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "residual_diff launch");
+  return PA_OK;
 }
 
 int pa_attn_chunks_noalloc(const void* q, const void* const* k_chunks, const void* const* v_chunks,

@@ -249,6 +249,34 @@ int pa_attn_merge(const void* o_parts, const float* lse_parts, int n_parts, void
                   int B, int H, int N, int d, void* stream);
 
 /*
+ * pa_residual_diff - First Block Cache's residual difference.
+ *
+ * diffusers "ParaAttention" guide, section "First Block Cache": the change of
+ * the first transformer block's residual output between two denoising steps
+ * approximates the change of the model's output, and the cached residuals
+ * are reused while it stays below a threshold (0.08 by default for FLUX).
+ * The guide gives no formula; this computes the relative L1 difference
+ *     out[0] = sum_i |cur_i - prev_i| / sum_i |prev_i|
+ * over the n elements (0 when both sums are 0, +inf when only the
+ * denominator is), accumulated in fp32 in a fixed order: the same inputs give
+ * the same bits on the same device.
+ *
+ * cur, prev  [n] bf16, device, 16-byte aligned                (inputs; may be the same buffer)
+ * out        [1] fp32, device, 4-byte aligned                 (output)
+ * n >= 1.
+ *
+ * Two launches on `stream`.  The block partials live in a small array the
+ * library reserves statically on each GPU: calls that overlap on the GPU
+ * (different streams, no ordering) race on it; calls ordered on one stream
+ * do not.
+ *
+ * Errors: PA_ERR_INVALID_ARG (null pointer, n < 1, out overlapping an input),
+ * PA_ERR_MISALIGNED, PA_ERR_CUDA (including pointers that are not device
+ * memory).
+ */
+int pa_residual_diff(const void* cur, const void* prev, long long n, float* out, void* stream);
+
+/*
  * pa_attn_chunks_noalloc - attention of Q over several K/V chunks, allocating
  * nothing.
  *

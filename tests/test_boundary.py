@@ -232,6 +232,15 @@ def test_quantize_and_fp8_dev_argument_checks(lib):
     assert call(d=64) == B.PA_ERR_UNSUPPORTED
 
 
+def test_residual_diff_argument_checks(lib):
+    rd = lib.pa_residual_diff
+    assert rd(0, A + MB, 16, A + 2 * MB, None) == B.PA_ERR_INVALID_ARG
+    assert rd(A, A + MB, 0, A + 2 * MB, None) == B.PA_ERR_INVALID_ARG
+    assert rd(A + 8, A + MB, 16, A + 2 * MB, None) == B.PA_ERR_MISALIGNED
+    assert rd(A, A + MB, 16, A + 2 * MB + 2, None) == B.PA_ERR_MISALIGNED
+    assert rd(A, A + MB, 1024, A + 64, None) == B.PA_ERR_INVALID_ARG     # out inside cur (2 KB)
+
+
 def test_plain_c_caller(lib, tmp_path):
     """A C program compiled with gcc against the header and linked to the
     library gets the documented status codes (no Python in between)."""
